@@ -1,0 +1,77 @@
+"""Host-side arithmetic pinned to the worked numbers the pages print, and the
+input recipe."""
+import math
+import os
+
+import numpy as np
+import torch
+
+from tiled_attention_20_b200 import inputs, perf
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+
+
+def _rows(name):
+    with open(os.path.join(GOLDEN, name)) as f:
+        return [l.split() for l in f if l.strip() and not l.startswith("#")]
+
+
+def test_wave_quantization_golden():
+    for side, tm, tn, tiles, sms, nwaves, last in _rows("wave_quantization.txt"):
+        side, tm, tn, tiles, sms, nwaves, last = map(int, (side, tm, tn, tiles, sms, nwaves, last))
+        t = perf.tile_count(side, side, tm, tn)
+        assert t == tiles
+        assert perf.waves(t, sms) == nwaves
+        assert t - (nwaves - 1) * sms == last
+
+
+def test_roofline_golden():
+    for flops, nbytes, bw, peak, inten, bound in _rows("roofline_example.txt"):
+        flops, nbytes, bw, peak, inten, bound = map(float, (flops, nbytes, bw, peak, inten, bound))
+        assert flops / nbytes == inten
+        assert perf.roofline_bound(peak, bw, flops / nbytes) == bound
+
+
+def test_gemm_cost_golden_and_attention_flops():
+    for M, K, N, flops, nbytes in _rows("gemm_cost.txt"):
+        M, K, N, flops, nbytes = map(int, (M, K, N, flops, nbytes))
+        assert 2 * M * K * N == flops
+        assert 2 * (M * K + K * N + M * N) == nbytes
+    # attention forward = two N x N x d GEMMs per head
+    B, H, N, d = 2, 32, 4096, 128
+    assert perf.attention_flops(B, H, N, d, False, False) == B * H * 2 * (2 * N * d * N)
+    assert perf.attention_flops(B, H, N, d, True, False) == B * H * 2 * N * d * N
+    assert perf.attention_flops(B, H, N, d, True, True) == 2.5 * B * H * 2 * N * d * N
+
+
+def test_inputs_seeded_and_bf16():
+    a = inputs.qkv_do(1, 2, 64, 64, seed=0)
+    b = inputs.qkv_do(1, 2, 64, 64, seed=0)
+    c = inputs.qkv_do(1, 2, 64, 64, seed=1)
+    for x, y in zip(a, b):
+        assert x.dtype == torch.bfloat16 and x.is_contiguous()
+        assert torch.equal(x, y)
+    assert not torch.equal(a[0], c[0])
+    # the first draw is torch.randn(fp32) rounded to bf16
+    g = torch.Generator().manual_seed(0)
+    ref = torch.randn((1, 2, 64, 64), generator=g).to(torch.bfloat16)
+    assert torch.equal(a[0], ref)
+
+
+def test_long_context_recipe():
+    N = 1000
+    q, k, v, dO = inputs.qkv_do(1, 2, N, 64, seed=0, dist="long_context")
+    n_big = math.ceil(0.01 * N)
+    for t in (q, k):
+        rms = t.float().pow(2).mean(dim=-1).sqrt()[0]  # [H, N]
+        for h in range(2):
+            big = (rms[h] > 12).sum().item()  # rows x8 have rms ~24, others ~3
+            assert big == n_big
+    assert abs(v.float().std().item() - 1.0) < 0.05
+    assert abs(dO.float().std().item() - 1.0) < 0.05
+
+
+def test_sweep_has_48_cases():
+    ws = inputs.sweep_workloads()
+    assert len(ws) == 48
+    assert len({w.name for w in ws}) == 48

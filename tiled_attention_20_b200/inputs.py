@@ -1,0 +1,91 @@
+"""Seeded synthetic inputs shared by the oracle tests, the GPU parity tests and
+the benchmark.
+
+This module holds no attention arithmetic: only random draws, the workload
+shapes, and bf16 rounding of the draws.  Draws happen on the CPU with a
+``torch.Generator`` so that both sides see bit-identical inputs.
+
+Recipe (one generator per call, seeded with ``seed``):
+
+1. ``torch.randn`` in fp32, in the order Q, K, V, dO, each [B, H, N, d].
+2. ``dist == "long_context"`` (the long-context workload): Q and K are scaled
+   by 3 (standard deviation 3), then, for each (b, h) in order, ceil(0.01 N)
+   query rows and then ceil(0.01 N) key rows, drawn without replacement with
+   ``torch.randperm`` from the same generator, are multiplied by 8.  V and dO
+   keep standard deviation 1.
+3. Everything is rounded to bf16 (round to nearest even).
+"""
+from __future__ import annotations
+
+import math
+from dataclasses import dataclass
+
+import torch
+
+
+@dataclass(frozen=True)
+class Workload:
+    """One attention problem: shape, mask, which passes, value distribution."""
+    name: str
+    B: int
+    H: int
+    N: int
+    d: int
+    causal: bool
+    backward: bool
+    dist: str = "normal"
+    seed: int = 0
+
+
+# The five workload families the method is measured and checked on.
+SMALL_FWD = Workload("fwd_nc_B1_H2_N256_d64", 1, 2, 256, 64, False, False)
+MID_NC = Workload("fwdbwd_nc_B4_H16_N1024_d64", 4, 16, 1024, 64, False, True)
+MID_C = Workload("fwdbwd_c_B4_H16_N1024_d64", 4, 16, 1024, 64, True, True)
+GPT_CAUSAL = Workload("fwdbwd_c_B2_H32_N4096_d128", 2, 32, 4096, 128, True, True)
+LONG_CONTEXT = Workload("fwdbwd_c_B1_H16_N16384_d128_lc", 1, 16, 16384, 128, True, True,
+                        dist="long_context")
+
+
+def sweep_workloads():
+    """The boundary / wave sweep: H=16, d in {64,128}, B in {1,8},
+    N in {1792,1793,2048,2049,4000,8192}, causal and not; fwd and bwd."""
+    out = []
+    for d in (64, 128):
+        for B in (1, 8):
+            for N in (1792, 1793, 2048, 2049, 4000, 8192):
+                for causal in (False, True):
+                    tag = "c" if causal else "nc"
+                    out.append(Workload(f"sweep_{tag}_B{B}_H16_N{N}_d{d}", B, 16, N, d,
+                                        causal, True))
+    return out
+
+
+def qkv_do(B: int, H: int, N: int, d: int, seed: int = 0, dist: str = "normal",
+           device: str | torch.device = "cpu"):
+    """(q, k, v, dO) as contiguous bf16 [B, H, N, d] tensors."""
+    g = torch.Generator(device="cpu").manual_seed(int(seed))
+    shape = (B, H, N, d)
+    q = torch.randn(shape, generator=g, dtype=torch.float32)
+    k = torch.randn(shape, generator=g, dtype=torch.float32)
+    v = torch.randn(shape, generator=g, dtype=torch.float32)
+    dO = torch.randn(shape, generator=g, dtype=torch.float32)
+    if dist == "long_context":
+        q.mul_(3.0)
+        k.mul_(3.0)
+        n_big = math.ceil(0.01 * N)
+        for b in range(B):
+            for h in range(H):
+                iq = torch.randperm(N, generator=g)[:n_big]
+                ik = torch.randperm(N, generator=g)[:n_big]
+                q[b, h, iq] *= 8.0
+                k[b, h, ik] *= 8.0
+    elif dist != "normal":
+        raise ValueError(f"unknown distribution {dist!r}")
+    out = tuple(t.to(torch.bfloat16).contiguous() for t in (q, k, v, dO))
+    if str(device) != "cpu":
+        out = tuple(t.to(device) for t in out)
+    return out
+
+
+def for_workload(w: Workload, device="cpu"):
+    return qkv_do(w.B, w.H, w.N, w.d, seed=w.seed, dist=w.dist, device=device)
