@@ -1,0 +1,124 @@
+/*
+ * fa.h -- C ABI of libfa: exact attention (forward and backward) on B200 (sm_100a).
+ *
+ * The operation ("第17讲 Tensor Core、HBM、SRAM 与 FlashAttention", §8.1 scaled
+ * dot-product attention; §8.2 the tiled flow; §8.3 online softmax):
+ *
+ *     O = softmax(scale * Q K^T [+ causal mask]) V
+ *
+ * evaluated tile by tile with an online softmax, so the N x N score and
+ * probability matrices never reach device memory.  The forward also writes
+ * the per-row log-sum-exp lse_i = ln sum_j exp(scale q_i.k_j) (natural log,
+ * over the visible keys), from which the backward recomputes the
+ * probabilities instead of storing them ("CS336 Lecture 5 · GPUs, TPUs"
+ * notes, section "FlashAttention 解析", item ② on recomputation).
+ *
+ * Conventions shared by every entry point:
+ *   - Tensors Q, K, V, O, dO, dQ, dK, dV are dense row-major [B, H, N, d]
+ *     (d contiguous, then N, then H, then B), bf16 unless stated.  lse and
+ *     the backward's D are [B, H, N] fp32.  Queries and keys share length N.
+ *   - causal != 0 means query i sees keys j <= i (top-left aligned).
+ *   - d must be 64 or 128.  N >= 1, B >= 1, H >= 1, B*H*N*d < 2^31.
+ *   - scale must be finite and >= 0 (1/sqrt(d) is the usual choice).
+ *   - Device pointers must be 16-byte aligned (lse and workspace: 16 bytes
+ *     too).  The caller owns every buffer: the library allocates, frees and
+ *     synchronises nothing; all work is enqueued on `stream` (0 = legacy
+ *     default stream) of the current device.
+ *   - Arguments are validated before anything is launched; on error nothing
+ *     is enqueued and a negative fa_status is returned.  No exception ever
+ *     crosses the ABI.
+ *   - Calls are thread-safe.  Two calls that run concurrently on the GPU must
+ *     not share output or workspace buffers.
+ *   - Results are deterministic for the forward.  The backward accumulates dQ
+ *     with floating-point atomics, so dQ may differ in the last bits between
+ *     runs (the pages note that tiled attention is not bit-identical to the
+ *     untiled computation, §8.4 of the first page).
+ */
+#ifndef FA_H_
+#define FA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct CUstream_st *fa_stream_t; /* same type as cudaStream_t */
+
+typedef enum {
+  FA_OK = 0,
+  FA_ERR_NULL = -1,           /* a required pointer is NULL */
+  FA_ERR_SHAPE = -2,          /* B, H or N < 1, or a tensor too large */
+  FA_ERR_UNSUPPORTED_D = -3,  /* d not in {64, 128} */
+  FA_ERR_ALIGN = -4,          /* a pointer is not 16-byte aligned */
+  FA_ERR_WORKSPACE = -5,      /* workspace smaller than fa_bwd_workspace_size */
+  FA_ERR_LAUNCH = -6,         /* the CUDA runtime rejected a launch or query */
+  FA_ERR_TIMEOUT = -7,        /* a device-side wait gave up (reported later) */
+  FA_ERR_DEVICE_ASSERT = -8,  /* a device-side consistency check failed */
+  FA_ERR_ARCH = -9,           /* the current device is not sm_100 */
+  FA_ERR_ARG = -10            /* scale negative or not finite; bad grad_dtype */
+} fa_status;
+
+/*
+ * Forward.
+ *   q, k, v : inputs, bf16 [B,H,N,d], device memory, read only.
+ *   o       : output, bf16 [B,H,N,d], device memory, written.
+ *   lse     : output, fp32 [B,H,N], device memory, written (natural log).
+ * Returns FA_OK once the kernel is enqueued.  Kernel-side failures (a bounded
+ * wait that timed out) are latched in a per-device status word that
+ * fa_check_device_errors() reads.
+ */
+int fa_fwd(const void *q, const void *k, const void *v, void *o, float *lse,
+           int B, int H, int N, int d, float scale, int causal,
+           fa_stream_t stream);
+
+/*
+ * Backward: gradients of L = sum(O * dO) for the forward above.  The
+ * formulas are not on the pages (they only say the backward recomputes the
+ * probabilities tile by tile); the library computes the exact gradient:
+ *     P_ij  = exp(scale q_i.k_j - lse_i)        (0 where masked)
+ *     D_i   = sum_c dO_ic O_ic
+ *     dV_j  = sum_i P_ij dO_i
+ *     dS_ij = P_ij (dO_i.v_j - D_i)
+ *     dQ_i  = scale sum_j dS_ij k_j,   dK_j = scale sum_i dS_ij q_i
+ *   q, k, v, o, dO : bf16 [B,H,N,d], device, read only (o and lse from fa_fwd
+ *                    with the same q, k, v, scale and causal).
+ *   lse            : fp32 [B,H,N], device, read only.
+ *   dq, dk, dv     : outputs [B,H,N,d], device, written; bf16 when
+ *                    grad_dtype == 0, fp32 when grad_dtype == 1.
+ *   workspace      : device scratch of at least fa_bwd_workspace_size(B,H,N,d)
+ *                    bytes, 16-byte aligned, owned by the caller; its contents
+ *                    on entry do not matter and on exit are unspecified.
+ */
+int fa_bwd(const void *q, const void *k, const void *v, const void *o,
+           const void *dO, const float *lse, void *dq, void *dk, void *dv,
+           int B, int H, int N, int d, float scale, int causal,
+           void *workspace, size_t workspace_bytes, int grad_dtype,
+           fa_stream_t stream);
+
+/* Bytes of scratch fa_bwd needs: an fp32 dQ accumulator [B,H,N,d] and the
+ * fp32 D vector [B,H,N], each rounded up to 256 bytes.  0 on invalid shapes. */
+size_t fa_bwd_workspace_size(int B, int H, int N, int d);
+
+/* Human-readable text for an fa_status value (static storage). */
+const char *fa_strerror(int status);
+
+/* Synchronises `stream`, then reads and clears the current device's status
+ * word that kernels set when a bounded wait gives up or a consistency check
+ * fails.  Returns FA_OK, FA_ERR_TIMEOUT, FA_ERR_DEVICE_ASSERT or
+ * FA_ERR_LAUNCH (a CUDA error is pending on the device). */
+int fa_check_device_errors(fa_stream_t stream);
+
+/* Number of persistent CTAs fa_fwd / fa_bwd launch for a problem on the
+ * current device (pass = 0 forward, 1 backward), and the number of work
+ * units they share; for the harness and its wave-quantization checks.
+ * Returns FA_OK or an error status (no launch happens). */
+int fa_launch_shape(int pass, int B, int H, int N, int d, int causal,
+                    int *ctas, int *work_units);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* FA_H_ */

@@ -1,0 +1,87 @@
+"""The C ABI without a GPU: the library loads, exports every symbol the header
+declares, and rejects bad arguments before touching the device."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import tiled_attention_20_b200.build as fa_build
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    fa_build.build()
+    import tiled_attention_20_b200.fa as fa
+    return fa.load()
+
+
+def _declared():
+    text = open(os.path.join(ROOT, "include", "fa.h")).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(fa_[a-z_0-9]+)\s*\(", text)))
+
+
+def test_exports_every_declared_symbol(lib):
+    names = _declared()
+    assert {"fa_fwd", "fa_bwd", "fa_bwd_workspace_size", "fa_strerror",
+            "fa_check_device_errors"} <= set(names)
+    for n in names:
+        assert hasattr(lib, n), n
+
+
+def test_strerror_covers_all_codes(lib):
+    import tiled_attention_20_b200.fa as fa
+    for code in fa.STATUS_NAMES:
+        assert fa.strerror(code) != "unknown status"
+    assert fa.strerror(12345) == "unknown status"
+
+
+def test_workspace_size(lib):
+    import tiled_attention_20_b200.fa as fa
+    ws = fa.workspace_size(2, 32, 4096, 128)
+    rows = 2 * 32 * 4096
+    assert ws >= rows * 128 * 4 + rows * 4 and ws % 256 == 0
+    assert fa.workspace_size(0, 1, 1, 64) == 0
+    assert fa.workspace_size(1, 1, 1, 96) == 0
+
+
+P = 0x10000  # a fake, 16-byte aligned "device pointer": validation fails before any use
+
+
+@pytest.mark.parametrize("args,code", [
+    ((0, P, P, P, P, 1, 1, 1, 64, 0.1, 0), -1),        # NULL q
+    ((P, P, P, P, P, 0, 1, 1, 64, 0.1, 0), -2),        # B = 0
+    ((P, P, P, P, P, 1, 1, 0, 64, 0.1, 0), -2),        # N = 0
+    ((P, P, P, P, P, 1, 1, 16, 96, 0.1, 0), -3),       # d = 96
+    ((P, P, P, P, P, 1024, 1024, 1024, 64, 0.1, 0), -2),  # too large
+    ((P + 2, P, P, P, P, 1, 1, 16, 64, 0.1, 0), -4),   # misaligned q
+    ((P, P, P, P, P, 1, 1, 16, 64, -1.0, 0), -10),     # negative scale
+    ((P, P, P, P, P, 1, 1, 16, 64, float("nan"), 0), -10),
+])
+def test_fwd_validation(lib, args, code):
+    assert lib.fa_fwd(*args, None) == code
+
+
+def test_bwd_validation(lib):
+    base = [P] * 9 + [1, 1, 16, 64, 0.1, 0, P, 1 << 20, 0, None]
+    assert lib.fa_bwd(*base[:15], 0, 1 << 20, 0, None) == -1          # NULL workspace
+    bad = list(base); bad[17] = 2
+    assert lib.fa_bwd(*bad) == -10                                     # grad_dtype
+    bad = list(base); bad[16] = 16
+    assert lib.fa_bwd(*bad) == -5                                      # workspace too small
+    bad = list(base); bad[12] = 32
+    assert lib.fa_bwd(*bad) == -3
+    bad = list(base); bad[6] = P + 8
+    assert lib.fa_bwd(*bad) == -4
+
+
+def test_no_device_means_launch_error_not_crash(lib):
+    """Valid arguments on a machine without a GPU: an error status, no crash."""
+    import torch
+    if torch.cuda.is_available():
+        pytest.skip("a GPU is present")
+    code = lib.fa_fwd(P, P, P, P, P, 1, 1, 16, 64, 0.125, 0, None)
+    assert code in (-6, -9)

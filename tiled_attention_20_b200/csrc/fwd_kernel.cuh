@@ -1,0 +1,434 @@
+// fwd_kernel.cuh -- attention forward on sm_100a.
+//
+// Computes O = softmax(scale Q K^T [+ causal]) V and lse per row, tile by tile
+// with the online softmax of "第17讲 Tensor Core、HBM、SRAM 与
+// FlashAttention" §8.3 (running max m, running sum l, rescale of the output
+// accumulator by e^{m - m'}, O = o / l at the end), following the tiled flow
+// of §8.2 of the same page: a Q tile is loaded once, K/V tiles are streamed
+// through shared memory, and scores and probabilities live only on chip.
+//
+// B200 mapping (one persistent CTA per SM, 12 warps):
+//   warp 0      TMA producer: Q tile pair once per work unit, then a K ring
+//               and a V ring of kStages slots each.
+//   warp 1      TMEM allocator and single-thread tcgen05.mma issuer.
+//   warps 4-7   softmax warpgroup 0: owns Q tile 0 (rows q0 .. q0+127).
+//   warps 8-11  softmax warpgroup 1: owns Q tile 1 (rows q0+128 .. q0+255).
+// TMEM (512 columns): S0 [0,128) S1 [128,256) O0 [256,256+D) O1 [256+D,256+2D).
+// P_i (bf16, packed in pairs) overwrites the first 64 columns of S_i and is
+// the A operand of O_i += P_i V straight from TMEM.  One thread owns one row,
+// so row max and row sum need no shuffles.
+//
+// A work unit is (b*H+h, pair of 128-row Q tiles); units are visited longest
+// first when causal, and CTAs stride through them (persistent grid of
+// min(units, SMs) CTAs), so no partial last wave of whole CTAs is left
+// (wave quantization, "CS336 Lecture 5 · GPUs, TPUs" notes, section
+// "波次量化").
+//
+// Causal masking is by tile skipping: Q tile i only visits key tiles up to
+// its diagonal, and only the diagonal tile (and a ragged last key tile) pays
+// for an element mask, which is a select to -inf (no divergent branches).
+//
+// The output rescale is lazy: the running max used for the exponentials is
+// only raised when a tile's maximum exceeds it by more than 2^8 (in the
+// exp2 domain), so most tiles skip the O read-modify-write.  The result is
+// unchanged because O and l are always scaled by the same reference.
+#pragma once
+#include "sm100.cuh"
+
+namespace fa {
+
+struct FwdParams {
+  __nv_bfloat16* o;
+  float* lse;
+  int BH;
+  int N;
+  int n_qt2;       // ceil(N / 256): Q tile pairs per head
+  int n_units;     // BH * n_qt2
+  float scale_log2;  // scale * log2(e)
+  int* status;
+};
+
+template <int D>
+struct FwdLayout {
+  static constexpr int kTileBytes = 128 * D * 2;
+  static constexpr int kStages = (D == 64) ? 4 : 2;
+  static constexpr int kQ0 = 0;
+  static constexpr int kQ1 = kTileBytes;
+  static constexpr int kK = 2 * kTileBytes;
+  static constexpr int kV = kK + kStages * kTileBytes;
+  static constexpr int kBar = kV + kStages * kTileBytes;
+  static constexpr int kBarBytes = 512;
+  static constexpr int kSmemBytes = kBar + kBarBytes + 1024;  // + manual 1024-B alignment
+};
+
+struct FwdBarriers {
+  uint64_t q_full, q_empty;
+  uint64_t k_full[4], k_empty[4], v_full[4], v_empty[4];
+  uint64_t s_full[2], p_full[2], o_full[2];
+  uint64_t mma_done;
+  uint32_t tmem_base;
+  int abort_flag;
+};
+
+struct FwdUnit {
+  int bh, q0, nk0, nk1;
+};
+
+template <bool CAUSAL>
+__device__ __forceinline__ FwdUnit fwd_decode(const FwdParams& p, int w) {
+  FwdUnit u;
+  const int idx = w / p.BH;
+  u.bh = w - idx * p.BH;
+  const int qt2 = CAUSAL ? (p.n_qt2 - 1 - idx) : idx;
+  u.q0 = qt2 * 256;
+  const int nkv = (p.N + 127) / 128;
+  u.nk0 = CAUSAL ? min(2 * qt2 + 1, nkv) : nkv;
+  u.nk1 = CAUSAL ? min(2 * qt2 + 2, nkv) : nkv;
+  return u;
+}
+
+// Wait on an mbarrier from one thread; false (and the CTA's abort flag set)
+// if the wait timed out or another role already aborted.
+__device__ __forceinline__ bool wait1(uint64_t* bar, uint32_t parity, FwdBarriers* b,
+                                      int* status) {
+  if (*(volatile int*)&b->abort_flag) return false;
+  if (mbar_wait(bar, parity, status)) return true;
+  *(volatile int*)&b->abort_flag = 1;
+  return false;
+}
+
+// The same from every lane of a warp, with a warp-uniform answer.
+__device__ __forceinline__ bool wait_warp(uint64_t* bar, uint32_t parity, FwdBarriers* b,
+                                          int* status) {
+  bool ok = !*(volatile int*)&b->abort_flag;
+  if (ok) ok = mbar_wait(bar, parity, status);
+  ok = __all_sync(0xffffffffu, ok);
+  if (!ok) *(volatile int*)&b->abort_flag = 1;
+  return ok;
+}
+
+// ---------------------------------------------------------------- producer
+template <int D, bool CAUSAL>
+__device__ void fwd_producer(const CUtensorMap* tm_q, const CUtensorMap* tm_k,
+                             const CUtensorMap* tm_v, const FwdParams& p, uint8_t* smem,
+                             FwdBarriers* b, int& kc, int& vc, int& units) {
+  using L = FwdLayout<D>;
+  constexpr int S = L::kStages;
+  for (int w = blockIdx.x; w < p.n_units; w += gridDim.x) {
+    const FwdUnit u = fwd_decode<CAUSAL>(p, w);
+    if (units > 0 && !wait1(&b->q_empty, (units - 1) & 1, b, p.status)) return;
+    mbar_arrive_expect_tx(&b->q_full, 2 * L::kTileBytes);
+    ++units;  // number of times q_full has been armed
+#pragma unroll
+    for (int c = 0; c < D / 64; ++c) {
+      tma_load_3d(smem + L::kQ0 + c * 16384, tm_q, &b->q_full, c * 64, u.q0, u.bh);
+      tma_load_3d(smem + L::kQ1 + c * 16384, tm_q, &b->q_full, c * 64, u.q0 + 128, u.bh);
+    }
+    const int nk = u.nk1;
+    for (int j = 0; j < nk; ++j) {
+      {
+        const int st = kc % S;
+        if (kc >= S && !wait1(&b->k_empty[st], ((kc / S) - 1) & 1, b, p.status)) return;
+        mbar_arrive_expect_tx(&b->k_full[st], L::kTileBytes);
+#pragma unroll
+        for (int c = 0; c < D / 64; ++c)
+          tma_load_3d(smem + L::kK + st * L::kTileBytes + c * 16384, tm_k, &b->k_full[st],
+                      c * 64, j * 128, u.bh);
+        ++kc;
+      }
+      {
+        const int st = vc % S;
+        if (vc >= S && !wait1(&b->v_empty[st], ((vc / S) - 1) & 1, b, p.status)) return;
+        mbar_arrive_expect_tx(&b->v_full[st], L::kTileBytes);
+#pragma unroll
+        for (int c = 0; c < D / 64; ++c)
+          tma_load_3d(smem + L::kV + st * L::kTileBytes + c * 16384, tm_v, &b->v_full[st],
+                      c * 64, j * 128, u.bh);
+        ++vc;
+      }
+    }
+  }
+}
+
+// ---------------------------------------------------------------- MMA issuer
+template <int D>
+__device__ __forceinline__ void issue_s(uint32_t tmem_s, uint32_t q_smem, uint32_t k_smem) {
+  constexpr uint32_t idesc = idesc_bf16_f32(128, 128, false, false);
+#pragma unroll
+  for (int kk = 0; kk < D / 16; ++kk) {
+    const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
+    mma_ss(tmem_s, sdesc_sw128(q_smem + off, 16, 1024), sdesc_sw128(k_smem + off, 16, 1024),
+           idesc, kk > 0 ? 1u : 0u);
+  }
+}
+
+template <int D>
+__device__ __forceinline__ void issue_pv(uint32_t tmem_o, uint32_t tmem_p, uint32_t v_smem,
+                                         bool accumulate) {
+  constexpr uint32_t idesc = idesc_bf16_f32(128, D, false, true);
+#pragma unroll
+  for (int kk = 0; kk < 8; ++kk) {
+    mma_ts(tmem_o, tmem_p + kk * 8, sdesc_sw128(v_smem + kk * 2048, 16384, 1024), idesc,
+           (accumulate || kk > 0) ? 1u : 0u);
+  }
+}
+
+template <int D, bool CAUSAL>
+__device__ void fwd_mma(const FwdParams& p, uint8_t* smem, FwdBarriers* b, uint32_t tmem) {
+  using L = FwdLayout<D>;
+  constexpr int S = L::kStages;
+  const uint32_t sb = smem_u32(smem);
+  const uint32_t tS[2] = {tmem + 0, tmem + 128};
+  const uint32_t tO[2] = {tmem + 256, tmem + 256 + D};
+  const uint32_t qs[2] = {sb + L::kQ0, sb + L::kQ1};
+  int qc = 0, kc = 0, vc = 0;
+  int pc[2] = {0, 0};
+  for (int w = blockIdx.x; w < p.n_units; w += gridDim.x) {
+    const FwdUnit u = fwd_decode<CAUSAL>(p, w);
+    const int nk0 = u.nk0, nk1 = u.nk1, nk = u.nk1;
+    if (!wait1(&b->q_full, qc & 1, b, p.status)) return;
+    ++qc;
+    tc_fence_after();
+    for (int j = 0; j < nk; ++j) {
+      const int ks = kc % S;
+      if (!wait1(&b->k_full[ks], (kc / S) & 1, b, p.status)) return;
+      tc_fence_after();
+      const uint32_t k_smem = sb + L::kK + ks * L::kTileBytes;
+      const int vs = vc % S;
+      const uint32_t v_smem = sb + L::kV + vs * L::kTileBytes;
+      if (j >= 1) {
+        if (!wait1(&b->v_full[vs], (vc / S) & 1, b, p.status)) return;
+        tc_fence_after();
+      }
+      if (j >= 1 && j - 1 < nk0) {
+        if (!wait1(&b->p_full[0], pc[0] & 1, b, p.status)) return;
+        ++pc[0];
+        tc_fence_after();
+        issue_pv<D>(tO[0], tS[0], v_smem, j - 1 > 0);
+        if (j - 1 == nk0 - 1) mma_commit(&b->o_full[0]);
+      }
+      if (j < nk0) {
+        issue_s<D>(tS[0], qs[0], k_smem);
+        mma_commit(&b->s_full[0]);
+      }
+      if (j >= 1 && j - 1 < nk1) {
+        if (!wait1(&b->p_full[1], pc[1] & 1, b, p.status)) return;
+        ++pc[1];
+        tc_fence_after();
+        issue_pv<D>(tO[1], tS[1], v_smem, j - 1 > 0);
+        if (j - 1 == nk1 - 1) mma_commit(&b->o_full[1]);
+      }
+      if (j >= 1) {
+        mma_commit(&b->v_empty[vs]);
+        ++vc;
+      }
+      if (j < nk1) {
+        issue_s<D>(tS[1], qs[1], k_smem);
+        mma_commit(&b->s_full[1]);
+      }
+      mma_commit(&b->k_empty[ks]);
+      ++kc;
+    }
+    mma_commit(&b->q_empty);
+    // P V for the last key tile.
+    const int vs = vc % S;
+    const uint32_t v_smem = sb + L::kV + vs * L::kTileBytes;
+    if (!wait1(&b->v_full[vs], (vc / S) & 1, b, p.status)) return;
+    tc_fence_after();
+    if (nk - 1 < nk0) {
+      if (!wait1(&b->p_full[0], pc[0] & 1, b, p.status)) return;
+      ++pc[0];
+      tc_fence_after();
+      issue_pv<D>(tO[0], tS[0], v_smem, nk - 1 > 0);
+      mma_commit(&b->o_full[0]);
+    }
+    if (nk - 1 < nk1) {
+      if (!wait1(&b->p_full[1], pc[1] & 1, b, p.status)) return;
+      ++pc[1];
+      tc_fence_after();
+      issue_pv<D>(tO[1], tS[1], v_smem, nk - 1 > 0);
+      mma_commit(&b->o_full[1]);
+    }
+    mma_commit(&b->v_empty[vs]);
+    ++vc;
+  }
+}
+
+// ---------------------------------------------------------------- softmax
+template <int D, bool CAUSAL>
+__device__ void fwd_softmax(const FwdParams& p, FwdBarriers* b, uint32_t tmem, int wg) {
+  const int t = threadIdx.x - 128 * (wg + 1);  // row within the Q tile == TMEM lane
+  const uint32_t lane_base = static_cast<uint32_t>(t & ~31) << 16;
+  const uint32_t tS = tmem + lane_base + (wg ? 128u : 0u);
+  const uint32_t tO = tmem + lane_base + 256u + wg * D;
+  const float sl2 = p.scale_log2;
+  const int N = p.N;
+  int sc = 0, oc = 0;
+  for (int w = blockIdx.x; w < p.n_units; w += gridDim.x) {
+    const FwdUnit u = fwd_decode<CAUSAL>(p, w);
+    const int nk = wg ? u.nk1 : u.nk0;
+    const int tile_row0 = u.q0 + wg * 128;
+    const int row = tile_row0 + t;
+    float m_used = -INFINITY;  // reference max (exp2 domain) of O and l
+    float l = 0.f;
+    for (int j = 0; j < nk; ++j) {
+      if (!wait_warp(&b->s_full[wg], sc & 1, b, p.status)) return;
+      ++sc;
+      tc_fence_after();
+      uint32_t r[128];
+      tmem_ld_x128(tS, r);
+      float* s = reinterpret_cast<float*>(r);
+      const int key0 = j * 128;
+      const bool need_mask = (key0 + 128 > N) || (CAUSAL && key0 + 127 > tile_row0);
+      if (need_mask) {
+        const int lim = CAUSAL ? min(row + 1, N) : N;  // keys < lim are visible
+#pragma unroll
+        for (int c = 0; c < 128; ++c) s[c] = (key0 + c < lim) ? s[c] : -INFINITY;
+      }
+      float mx[8];
+#pragma unroll
+      for (int i = 0; i < 8; ++i) mx[i] = s[i];
+#pragma unroll
+      for (int c = 8; c < 128; ++c) mx[c & 7] = fmaxf(mx[c & 7], s[c]);
+      float m_tile = fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])),
+                           fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7])));
+      m_tile *= sl2;
+      const bool need = m_tile > m_used + 8.0f;
+      if (__any_sync(0xffffffffu, need)) {
+        const float m_new = fmaxf(m_used, m_tile);
+        const float alpha = (m_new == -INFINITY) ? 1.f : ex2_approx(m_used - m_new);
+        l *= alpha;
+        if (j > 0) {
+#pragma unroll
+          for (int c0 = 0; c0 < D; c0 += 32) {
+            uint32_t o[32];
+            tmem_ld_x32(tO + c0, o);
+#pragma unroll
+            for (int c = 0; c < 32; ++c) o[c] = __float_as_uint(__uint_as_float(o[c]) * alpha);
+            tmem_st_x32(tO + c0, o);
+          }
+        }
+        m_used = m_new;
+      }
+      const float mb = (m_used == -INFINITY) ? 0.f : m_used;
+      float rs[4] = {0.f, 0.f, 0.f, 0.f};
+      uint32_t pk[64];
+#pragma unroll
+      for (int c = 0; c < 128; c += 2) {
+        const float p0 = ex2_approx(fmaf(s[c], sl2, -mb));
+        const float p1 = ex2_approx(fmaf(s[c + 1], sl2, -mb));
+        rs[(c >> 1) & 3] += p0 + p1;
+        pk[c >> 1] = pack_bf16x2(p0, p1);
+      }
+      l += (rs[0] + rs[1]) + (rs[2] + rs[3]);
+      tmem_st_x32(tS, pk);
+      tmem_st_x32(tS + 32, pk + 32);
+      tmem_st_wait();
+      tc_fence_before();
+      mbar_arrive(&b->p_full[wg]);
+    }
+    // Epilogue: O = o / l, lse = (m + log2 l) ln 2.
+    if (!wait_warp(&b->o_full[wg], oc & 1, b, p.status)) return;
+    ++oc;
+    tc_fence_after();
+    const float inv_l = 1.f / l;
+    const bool valid = row < N;
+    __nv_bfloat16* orow = p.o + (static_cast<size_t>(u.bh) * N + row) * D;
+#pragma unroll
+    for (int c0 = 0; c0 < D; c0 += 32) {
+      uint32_t o[32];
+      tmem_ld_x32(tO + c0, o);
+      uint32_t pkd[16];
+#pragma unroll
+      for (int c = 0; c < 16; ++c)
+        pkd[c] = pack_bf16x2(__uint_as_float(o[2 * c]) * inv_l, __uint_as_float(o[2 * c + 1]) * inv_l);
+      if (valid) {
+        uint4* dst = reinterpret_cast<uint4*>(orow + c0);
+#pragma unroll
+        for (int v = 0; v < 4; ++v)
+          dst[v] = make_uint4(pkd[4 * v], pkd[4 * v + 1], pkd[4 * v + 2], pkd[4 * v + 3]);
+      }
+    }
+    if (valid) p.lse[static_cast<size_t>(u.bh) * N + row] = (m_used + __log2f(l)) * 0.69314718055994531f;
+  }
+}
+
+// ---------------------------------------------------------------- kernel
+template <int D, bool CAUSAL>
+__global__ void __launch_bounds__(384, 1)
+    fa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                  const __grid_constant__ CUtensorMap tm_v, const FwdParams p) {
+  using L = FwdLayout<D>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~static_cast<uintptr_t>(1023));
+  FwdBarriers* b = reinterpret_cast<FwdBarriers*>(smem + L::kBar);
+  const int warp = threadIdx.x >> 5;
+
+  if (threadIdx.x == 0) {
+    mbar_init(&b->q_full, 1);
+    mbar_init(&b->q_empty, 1);
+    for (int i = 0; i < L::kStages; ++i) {
+      mbar_init(&b->k_full[i], 1);
+      mbar_init(&b->k_empty[i], 1);
+      mbar_init(&b->v_full[i], 1);
+      mbar_init(&b->v_empty[i], 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&b->s_full[i], 1);
+      mbar_init(&b->p_full[i], 128);
+      mbar_init(&b->o_full[i], 1);
+    }
+    mbar_init(&b->mma_done, 1);
+    b->abort_flag = 0;
+    fence_barrier_init();
+  }
+  if (warp == 0 && lane_id() == 0) {
+    prefetch_tmap(&tm_q);
+    prefetch_tmap(&tm_k);
+    prefetch_tmap(&tm_v);
+  }
+  if (warp == 1) {
+    tmem_alloc(&b->tmem_base, 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = b->tmem_base;
+
+  if (warp == 0) {
+    if (lane_id() == 0) {
+      int kc = 0, vc = 0, units = 0;
+      fwd_producer<D, CAUSAL>(&tm_q, &tm_k, &tm_v, p, smem, b, kc, vc, units);
+      // Wait for every TMA load this thread armed (all long complete on the
+      // normal path) so no copy is in flight when the CTA exits.
+      constexpr int S = L::kStages;
+      if (units > 0) mbar_wait(&b->q_full, (units - 1) & 1, p.status);
+      for (int st = 0; st < S; ++st) {
+        const int nk = kc / S + (st < kc % S ? 1 : 0);
+        const int nv = vc / S + (st < vc % S ? 1 : 0);
+        if (nk > 0) mbar_wait(&b->k_full[st], (nk - 1) & 1, p.status);
+        if (nv > 0) mbar_wait(&b->v_full[st], (nv - 1) & 1, p.status);
+      }
+    }
+    __syncwarp();
+  } else if (warp == 1) {
+    if (lane_id() == 0) {
+      fwd_mma<D, CAUSAL>(p, smem, b, tmem);
+      // Drain every MMA this thread issued before TMEM is released.
+      mma_commit(&b->mma_done);
+      mbar_wait(&b->mma_done, 0, p.status);
+    }
+    __syncwarp();
+  } else if (warp >= 4) {
+    fwd_softmax<D, CAUSAL>(p, b, tmem, (warp - 4) >> 2);
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 1) tmem_dealloc(tmem, 512);
+}
+
+}  // namespace fa

@@ -1,0 +1,157 @@
+"""Python binding of libfa (include/fa.h): argument marshalling only.
+
+Every step of the attention forward and backward runs in the CUDA kernels
+behind the C ABI; this module checks tensor properties, allocates outputs
+with PyTorch (device memory is plumbing) and passes raw pointers plus the
+current CUDA stream.  There is no CPU fallback: if libfa.so cannot be loaded,
+every call raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import math
+import os
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libfa.so")
+
+FA_OK = 0
+STATUS_NAMES = {
+    0: "FA_OK", -1: "FA_ERR_NULL", -2: "FA_ERR_SHAPE", -3: "FA_ERR_UNSUPPORTED_D",
+    -4: "FA_ERR_ALIGN", -5: "FA_ERR_WORKSPACE", -6: "FA_ERR_LAUNCH", -7: "FA_ERR_TIMEOUT",
+    -8: "FA_ERR_DEVICE_ASSERT", -9: "FA_ERR_ARCH", -10: "FA_ERR_ARG",
+}
+
+EXPORTED = ["fa_fwd", "fa_bwd", "fa_bwd_workspace_size", "fa_strerror",
+            "fa_check_device_errors", "fa_launch_shape"]
+
+
+class FAError(RuntimeError):
+    def __init__(self, status: int, what: str):
+        self.status = status
+        super().__init__(f"{what}: {STATUS_NAMES.get(status, status)} ({strerror(status)})")
+
+
+_lib = None
+_vp, _i, _f, _sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_size_t
+
+
+def load(path: str = LIB_PATH):
+    """Load libfa.so and declare its signatures.  Raises if it is missing."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(path):
+            raise RuntimeError(
+                f"libfa.so not found at {path}: build it with "
+                "`python -m tiled_attention_20_b200.build` (there is no fallback)")
+        lib = ctypes.CDLL(path)
+        lib.fa_fwd.argtypes = [_vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _f, _i, _vp]
+        lib.fa_fwd.restype = _i
+        lib.fa_bwd.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp,
+                               _i, _i, _i, _i, _f, _i, _vp, _sz, _i, _vp]
+        lib.fa_bwd.restype = _i
+        lib.fa_bwd_workspace_size.argtypes = [_i, _i, _i, _i]
+        lib.fa_bwd_workspace_size.restype = _sz
+        lib.fa_strerror.argtypes = [_i]
+        lib.fa_strerror.restype = ctypes.c_char_p
+        lib.fa_check_device_errors.argtypes = [_vp]
+        lib.fa_check_device_errors.restype = _i
+        lib.fa_launch_shape.argtypes = [_i, _i, _i, _i, _i, _i,
+                                        ctypes.POINTER(_i), ctypes.POINTER(_i)]
+        lib.fa_launch_shape.restype = _i
+        _lib = lib
+    return _lib
+
+
+def strerror(status: int) -> str:
+    return load().fa_strerror(int(status)).decode()
+
+
+def _check(status: int, what: str):
+    if status != FA_OK:
+        raise FAError(status, what)
+
+
+def _stream(device) -> int:
+    return torch.cuda.current_stream(device).cuda_stream
+
+
+def _check_qkv(*ts):
+    q = ts[0]
+    if q.dim() != 4:
+        raise ValueError("expected [B, H, N, d] tensors")
+    for t in ts:
+        if not t.is_cuda:
+            raise ValueError("tensors must be on a CUDA device (no CPU fallback)")
+        if t.dtype != torch.bfloat16:
+            raise ValueError("inputs must be bf16")
+        if t.shape != q.shape:
+            raise ValueError("all inputs must share the shape [B, H, N, d]")
+        if not t.is_contiguous():
+            raise ValueError("inputs must be contiguous")
+        if t.device != q.device:
+            raise ValueError("inputs must be on one device")
+
+
+def default_scale(d: int) -> float:
+    return 1.0 / math.sqrt(d)
+
+
+def fwd(q, k, v, scale=None, causal=False, out=None, lse=None):
+    """O [B,H,N,d] bf16 and lse [B,H,N] fp32 (natural log)."""
+    _check_qkv(q, k, v)
+    B, H, N, d = q.shape
+    scale = default_scale(d) if scale is None else float(scale)
+    if out is None:
+        out = torch.empty_like(q)
+    if lse is None:
+        lse = torch.empty((B, H, N), dtype=torch.float32, device=q.device)
+    with torch.cuda.device(q.device):
+        st = load().fa_fwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(),
+                           lse.data_ptr(), B, H, N, d, scale, int(bool(causal)), _stream(q.device))
+    _check(st, "fa_fwd")
+    return out, lse
+
+
+def workspace_size(B, H, N, d) -> int:
+    return int(load().fa_bwd_workspace_size(B, H, N, d))
+
+
+def bwd(q, k, v, o, dO, lse, scale=None, causal=False, grad_dtype=torch.bfloat16,
+        workspace=None, dq=None, dk=None, dv=None):
+    """dQ, dK, dV [B,H,N,d] (bf16 or fp32) for the forward that produced o, lse."""
+    _check_qkv(q, k, v, o, dO)
+    B, H, N, d = q.shape
+    if lse.dtype != torch.float32 or tuple(lse.shape) != (B, H, N) or not lse.is_contiguous():
+        raise ValueError("lse must be contiguous fp32 [B, H, N]")
+    scale = default_scale(d) if scale is None else float(scale)
+    gd = {torch.bfloat16: 0, torch.float32: 1}[grad_dtype]
+    ws_bytes = workspace_size(B, H, N, d)
+    if workspace is None:
+        workspace = torch.empty(max(ws_bytes, 16), dtype=torch.uint8, device=q.device)
+    dq = torch.empty(q.shape, dtype=grad_dtype, device=q.device) if dq is None else dq
+    dk = torch.empty(q.shape, dtype=grad_dtype, device=q.device) if dk is None else dk
+    dv = torch.empty(q.shape, dtype=grad_dtype, device=q.device) if dv is None else dv
+    with torch.cuda.device(q.device):
+        st = load().fa_bwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(),
+                           dO.data_ptr(), lse.data_ptr(), dq.data_ptr(), dk.data_ptr(),
+                           dv.data_ptr(), B, H, N, d, scale, int(bool(causal)),
+                           workspace.data_ptr(), workspace.numel(), gd, _stream(q.device))
+    _check(st, "fa_bwd")
+    return dq, dk, dv
+
+
+def check_device_errors(device=None) -> None:
+    """Synchronise and raise if a kernel latched a device-side error."""
+    device = torch.cuda.current_device() if device is None else device
+    with torch.cuda.device(device):
+        _check(load().fa_check_device_errors(_stream(device)), "device status")
+
+
+def launch_shape(pass_: int, B, H, N, d, causal=False):
+    ctas, units = _i(0), _i(0)
+    _check(load().fa_launch_shape(pass_, B, H, N, d, int(bool(causal)), ctypes.byref(ctas),
+                                  ctypes.byref(units)), "fa_launch_shape")
+    return ctas.value, units.value
