@@ -1,0 +1,394 @@
+#!/usr/bin/env python
+"""Benchmark of exact attention forward + backward on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+One step is one pass of the whole hot path, forward (fa_fwd) then backward
+(fa_bwd), over the GPT-style causal workload B=2, H=32, N=4096, d=128 in bf16
+(synthetic seeded inputs).  Throughput counts 4*B*H*N^2*d FLOPs for the
+forward, halved when causal, and 2.5x that for the backward.
+
+Timing follows "第17讲 Tensor Core、HBM、SRAM 与 FlashAttention" §10.1-10.2:
+warm-up first, CUDA events on the launching stream with a synchronize on both
+sides, fixed shapes and dtypes, and a check of the outputs before timing.  The
+inputs and outputs of one step (about 0.6 GB) exceed the 126 MB L2, so no
+flush is needed between steps.
+
+Under torchrun (N > 1) every rank runs the same workload on its own GPU
+(heads are independent: weak scaling, no collective on the data path); the
+step time is the maximum over ranks and the value is all ranks' FLOPs divided
+by it.  Rank 0 prints one JSON line.
+
+--impl reference times the fp64 CPU oracle (the reference arm) on a bounded
+sample of the same workload, on the host cores.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import torch  # noqa: E402
+
+from tiled_attention_20_b200 import inputs, perf  # noqa: E402
+
+WORKLOAD = inputs.GPT_CAUSAL
+METRIC = "attention fwd+bwd TFLOP/s (bf16, causal, N=4096 d=128) and % of dense BF16 peak"
+UNIT = "TFLOP/s"
+KERNEL_SOURCES = ["fwd_kernel.cuh", "bwd_kernel.cuh", "sm100.cuh", "fa_api.cu"]
+
+
+def parse_args():
+    ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=500)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--e2e-steps", type=int, default=10)
+    ap.add_argument("--cpu-seconds", type=float, default=10.0,
+                    help="target CPU time of the oracle baseline sample")
+    ap.add_argument("--no-cpu-baseline", action="store_true",
+                    help="skip the CPU oracle leg (used for profiler runs)")
+    ap.add_argument("--no-e2e", action="store_true", help="skip the host-buffer leg (profiler runs)")
+    return ap.parse_args()
+
+
+def workload_config(w=WORKLOAD, extra=None):
+    cfg = {"workload": w.name, "B": w.B, "H": w.H, "N": w.N, "d": w.d, "causal": w.causal,
+           "passes": "fwd+bwd", "dist": w.dist, "seed": w.seed,
+           "l2": "inputs_exceed_l2 (no flush)"}
+    if extra:
+        cfg.update(extra)
+    return cfg
+
+
+def step_flops(w=WORKLOAD) -> float:
+    return (perf.attention_flops(w.B, w.H, w.N, w.d, w.causal, False) +
+            perf.attention_flops(w.B, w.H, w.N, w.d, w.causal, True))
+
+
+def measured_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            return json.load(f), "measured"
+    except OSError:
+        return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}, "fallback"
+
+
+def kernel_source_hash() -> str:
+    h = hashlib.sha256()
+    for name in KERNEL_SOURCES:
+        with open(os.path.join(ROOT, "tiled_attention_20_b200", "csrc", name), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def profiled_traffic(kernel: str):
+    """DRAM bytes per launch of `kernel` from the committed ncu summary, if it
+    was captured from the current kernel sources; else None."""
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    try:
+        with open(path) as f:
+            rec = json.load(f)
+    except (OSError, ValueError):
+        return None
+    ent = rec.get(kernel)
+    if not ent or ent.get("source_hash") != kernel_source_hash():
+        return None
+    return ent.get("dram_bytes_per_launch")
+
+
+# ---------------------------------------------------------------- clocks
+class ClockSampler:
+    """nvidia-smi samples of SM clock and throttle reasons every 200 ms."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.t0 = self.t1 = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-i", str(self.gpu), "-lms", "200"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+
+    def mark(self, which):
+        setattr(self, which, time.time())
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        time.sleep(0.25)
+        self.proc.terminate()
+        out, _ = self.proc.communicate(timeout=10)
+        rows = [r.split(", ") for r in out.strip().splitlines() if r.count(",") >= 8]
+        sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
+        mx = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i in range(4) if r[5 + i].strip() == "Active"})
+        # keep samples taken under load (clock above idle) when there are any
+        busy = [s for s in sm if s > 600] or sm
+        return {"sm_mhz": statistics.median(busy) if busy else None,
+                "sm_max_mhz": max(mx) if mx else None, "reasons": reasons,
+                "samples": len(rows)}
+
+
+# ---------------------------------------------------------------- CPU oracle
+def cpu_oracle_rate(q, k, v, dO, w, seconds: float):
+    """The oracle (fp64, as it stands) on whole heads of the workload until
+    `seconds` of wall time have passed; returns (TFLOP/s, heads, cores, s)."""
+    import oracle  # the benchmark's CPU-baseline leg is one of the oracle's permitted users
+    t0 = time.time()
+    heads = 0
+    total = w.B * w.H
+    while heads < total:
+        b, h = divmod(heads, w.H)
+        sl = lambda t: t[b:b + 1, h:h + 1]
+        oracle.fwd(sl(q), sl(k), sl(v), causal=w.causal)
+        oracle.bwd(sl(q), sl(k), sl(v), sl(dO), causal=w.causal)
+        heads += 1
+        if time.time() - t0 >= seconds:
+            break
+    el = time.time() - t0
+    fl = (perf.attention_flops(1, 1, w.N, w.d, w.causal, False) +
+          perf.attention_flops(1, 1, w.N, w.d, w.causal, True)) * heads
+    return fl / el / 1e12, heads, oracle.num_threads(), el
+
+
+def run_reference(args, rank, world):
+    """Reference arm: the fp64 oracle on the host cores, each step a bounded
+    sample (one head, truncated to N' query/key rows so that all K + W steps
+    end within about two minutes) of the benchmark workload."""
+    if rank != 0:
+        return
+    import oracle
+    w = WORKLOAD
+    q, k, v, dO = inputs.for_workload(w)
+    budget = 120.0 / max(1, args.steps + args.warmup)
+
+    def sample_step(n):
+        sl = lambda t: t[0:1, 0:1, :n].contiguous()
+        t0 = time.time()
+        oracle.fwd(sl(q), sl(k), sl(v), causal=w.causal)
+        oracle.bwd(sl(q), sl(k), sl(v), sl(dO), causal=w.causal)
+        return time.time() - t0
+
+    t_cal = sample_step(512)
+    n = int(512 * math.sqrt(max(budget, 1e-3) / max(t_cal, 1e-6)))
+    n = max(128, min(w.N, n // 64 * 64))
+    for _ in range(args.warmup):
+        sample_step(n)
+    t0 = time.time()
+    for _ in range(args.steps):
+        sample_step(n)
+    el = time.time() - t0
+    fl = (perf.attention_flops(1, 1, n, w.d, w.causal, False) +
+          perf.attention_flops(1, 1, n, w.d, w.causal, True))
+    value = fl * args.steps / el / 1e12
+    sample = f"one head (b=0,h=0) truncated to N'={n} rows, fwd+bwd per step, fp64"
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": el / args.steps * 1e3,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic", "config": workload_config(w, {"sample_N": n}),
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": oracle.num_threads(),
+                         "kind": "oracle", "sample": sample},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+# ---------------------------------------------------------------- our arm
+def run_ours(args, rank, world, local_rank, dist):
+    import tiled_attention_20_b200.fa as fa
+    from tiled_attention_20_b200 import build as fa_build
+
+    if rank == 0 or world == 1:
+        fa_build.build()
+    if world > 1:
+        dist.barrier()
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    w = WORKLOAD
+    q_h, k_h, v_h, dO_h = inputs.qkv_do(w.B, w.H, w.N, w.d, seed=w.seed + rank, dist=w.dist)
+    q, k, v, dO = (t.to(dev) for t in (q_h, k_h, v_h, dO_h))
+    o = torch.empty_like(q)
+    lse = torch.empty((w.B, w.H, w.N), dtype=torch.float32, device=dev)
+    dq, dk, dv = (torch.empty_like(q) for _ in range(3))
+    ws = torch.empty(fa.workspace_size(w.B, w.H, w.N, w.d), dtype=torch.uint8, device=dev)
+
+    def step():
+        fa.fwd(q, k, v, causal=w.causal, out=o, lse=lse)
+        fa.bwd(q, k, v, o, dO, lse, causal=w.causal, workspace=ws, dq=dq, dk=dk, dv=dv)
+
+    # Output check before timing (no oracle here): finite results, and row 0
+    # of a causal head sees only key 0, so O_0 must equal V_0 bit for bit.
+    step()
+    fa.check_device_errors(dev)
+    for t in (o, lse, dq, dk, dv):
+        if not torch.isfinite(t).all():
+            raise RuntimeError("non-finite output")
+    if w.causal and not torch.equal(o[:, :, 0], v[:, :, 0]):
+        raise RuntimeError("causal row 0 does not equal V_0")
+
+    for _ in range(max(0, args.warmup - 1)):
+        step()
+    stream = torch.cuda.current_stream(dev)
+    sampler = ClockSampler(dev.index if world == 1 else local_rank)
+    sampler.start()
+    time.sleep(0.4)  # let the sampler come up
+    # keep the GPU busy while the sampler starts, outside the timed region
+    for _ in range(max(3, args.warmup)):
+        step()
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize(dev)
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    fa.trace_start()
+    e0.record(stream)
+    for _ in range(args.steps):
+        step()
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    traced = fa.trace_stop()
+    if world > 1:
+        dist.barrier()
+    clocks = sampler.stop()
+    fa.check_device_errors(dev)
+    ms = e0.elapsed_time(e1) / args.steps
+    if world > 1:
+        t = torch.tensor([ms], device=dev, dtype=torch.float64)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms = float(t.item())
+    flops = step_flops(w)
+    value = flops * world / (ms * 1e-3) / 1e12
+
+    # dominant kernel by traced time
+    dom = max(traced.items(), key=lambda kv: kv[1][1])
+    dom_name, (dom_launches, dom_ms) = dom
+    per_launch_ms = dom_ms / dom_launches
+    kernel_flops = {
+        "fa_fwd_kernel": perf.attention_flops(w.B, w.H, w.N, w.d, w.causal, False),
+        "fa_bwd_kernel": perf.attention_flops(w.B, w.H, w.N, w.d, w.causal, True),
+    }
+    peaks, peaks_src = measured_peaks()
+    if dom_name in kernel_flops:
+        achieved = kernel_flops[dom_name] / (per_launch_ms * 1e-3) / 1e12
+        roof = {"bound": "tensor", "achieved": achieved, "peak": peaks["bf16_tflops"],
+                "unit": "TFLOP/s", "frac": achieved / peaks["bf16_tflops"],
+                "traffic": profiled_traffic(dom_name), "kernel": dom_name,
+                "peak_source": f"{peaks_src} bf16_tflops (burst)",
+                "frac_of_sustained": achieved / peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"]),
+                "launch_ms": per_launch_ms}
+    else:  # a memory-bound helper dominating would be a regression worth seeing
+        roof = {"bound": "hbm", "achieved": None, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                "frac": None, "traffic": None, "kernel": dom_name}
+    kernels = {name: {"launches": n, "avg_ms": t / n} for name, (n, t) in traced.items()}
+    gpu_launches = sum(n for n, _ in traced.values())
+
+    # end to end through the public API with host buffers
+    e2e = None
+    if not args.no_e2e:
+        pin = lambda t: t.pin_memory()
+        hq, hk, hv, hdO = (pin(t) for t in (q_h, k_h, v_h, dO_h))
+        ho = torch.empty(q_h.shape, dtype=torch.bfloat16).pin_memory()
+        hlse = torch.empty((w.B, w.H, w.N), dtype=torch.float32).pin_memory()
+        hdq, hdk, hdv = (torch.empty(q_h.shape, dtype=torch.bfloat16).pin_memory() for _ in range(3))
+
+        def e2e_step():
+            q.copy_(hq, non_blocking=True)
+            k.copy_(hk, non_blocking=True)
+            v.copy_(hv, non_blocking=True)
+            dO.copy_(hdO, non_blocking=True)
+            step()
+            ho.copy_(o, non_blocking=True)
+            hlse.copy_(lse, non_blocking=True)
+            hdq.copy_(dq, non_blocking=True)
+            hdk.copy_(dk, non_blocking=True)
+            hdv.copy_(dv, non_blocking=True)
+
+        e2e_step()
+        torch.cuda.synchronize(dev)
+        if world > 1:
+            dist.barrier()
+        n_e2e = max(1, args.e2e_steps)
+        e0.record(stream)
+        for _ in range(n_e2e):
+            e2e_step()
+        e1.record(stream)
+        torch.cuda.synchronize(dev)
+        ms_e2e = e0.elapsed_time(e1) / n_e2e
+        if world > 1:
+            t = torch.tensor([ms_e2e], device=dev, dtype=torch.float64)
+            dist.all_reduce(t, op=dist.ReduceOp.MAX)
+            ms_e2e = float(t.item())
+        nb = lambda *ts: sum(t.numel() * t.element_size() for t in ts)
+        e2e = {"value": flops * world / (ms_e2e * 1e-3) / 1e12, "unit": UNIT,
+               "h2d_bytes_per_step": nb(hq, hk, hv, hdO),
+               "d2h_bytes_per_step": nb(ho, hlse, hdq, hdk, hdv), "steps": n_e2e,
+               "ms_per_step": ms_e2e, "api": "tiled_attention_20_b200.fa.fwd/bwd (C ABI)"}
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        rate, heads, cores, el = cpu_oracle_rate(q_h, k_h, v_h, dO_h, w, args.cpu_seconds)
+        cpu = {"value": rate, "unit": UNIT, "cores": cores, "kind": "oracle",
+               "sample": f"{heads} of {w.B * w.H} heads of the workload, fwd+bwd in fp64, "
+                         f"{el:.1f} s wall"}
+
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "bf16", "data": "synthetic",
+            "config": workload_config(w, {"parallelism": f"heads replicated per GPU x{world}"}),
+            "pct_of_peak": value / world / peaks["bf16_tflops"],
+            "roofline": roof, "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": gpu_launches,
+            "kernels": kernels, "clocks": clocks,
+        }
+        print(json.dumps(line), flush=True)
+
+
+def main():
+    args = parse_args()
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        run_reference(args, rank, world)
+        return
+    dist = None
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        torch.cuda.set_device(local_rank)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300))
+    try:
+        run_ours(args, rank, world, local_rank, dist)
+    finally:
+        if dist is not None:
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

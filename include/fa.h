@@ -29,10 +29,11 @@
  *     crosses the ABI.
  *   - Calls are thread-safe.  Two calls that run concurrently on the GPU must
  *     not share output or workspace buffers.
- *   - Results are deterministic for the forward.  The backward accumulates dQ
- *     with floating-point atomics, so dQ may differ in the last bits between
- *     runs (the pages note that tiled attention is not bit-identical to the
- *     untiled computation, §8.4 of the first page).
+ *   - Results are deterministic for the forward, dK and dV.  The backward
+ *     sums the per-block dQ contributions with fp32 reduce-add copies whose
+ *     order varies, so dQ may differ in the last bits between runs (the
+ *     pages note that tiled attention is not bit-identical to the untiled
+ *     computation, §8.4 of the first page).
  */
 #ifndef FA_H_
 #define FA_H_
@@ -97,8 +98,10 @@ int fa_bwd(const void *q, const void *k, const void *v, const void *o,
            void *workspace, size_t workspace_bytes, int grad_dtype,
            fa_stream_t stream);
 
-/* Bytes of scratch fa_bwd needs: an fp32 dQ accumulator [B,H,N,d] and the
- * fp32 D vector [B,H,N], each rounded up to 256 bytes.  0 on invalid shapes. */
+/* Bytes of scratch fa_bwd needs: an fp32 dQ accumulator [B,H,N,d], then
+ * lse * log2(e) and D = rowsum(dO * O) as fp32 [B,H,Npad] with Npad = N
+ * rounded up to 64, each rounded up to 256 bytes, then 256 bytes for the
+ * work-unit counter of the dynamic scheduler.  0 on invalid shapes. */
 size_t fa_bwd_workspace_size(int B, int H, int N, int d);
 
 /* Human-readable text for an fa_status value (static storage). */
@@ -116,6 +119,22 @@ int fa_check_device_errors(fa_stream_t stream);
  * Returns FA_OK or an error status (no launch happens). */
 int fa_launch_shape(int pass, int B, int H, int N, int d, int causal,
                     int *ctas, int *work_units);
+
+/*
+ * Opt-in per-kernel timing with CUDA events (a tracing aid; off by default).
+ * After fa_trace_start(), every kernel the library enqueues, on any stream of
+ * any device, is bracketed by two CUDA events recorded on its launch stream,
+ * until fa_trace_stop().  fa_trace_stop() waits for those events and fills,
+ * for each kernel id k < n_kernels, launches[k] and total_ms[k] (summed event
+ * durations).  Kernel ids: 0 forward, 1 backward preprocess, 2 backward main,
+ * 3 dQ conversion (fa_trace_kernel_name gives the kernel's name).  The
+ * library creates the events on first use and reuses them afterwards; event
+ * records add a few microseconds per launch.  fa_trace_start() discards a
+ * previous unfinished record.
+ */
+int fa_trace_start(void);
+int fa_trace_stop(int n_kernels, int *launches, double *total_ms);
+const char *fa_trace_kernel_name(int kernel);
 
 #ifdef __cplusplus
 }

@@ -29,5 +29,18 @@ def assert_close(name, gpu, ref, tol=None, ctx=""):
     return err
 
 
+def assert_close_scaled(name, gpu, ref, tol=None, ctx=""):
+    """Max-abs error bounded by tol * max(1, max|ref|).  Used where the
+    gradients are not unit-scale (a larger softmax scale, logits in the
+    hundreds): bf16 operand rounding is relative (2^-9), so the error of an
+    entry grows with the magnitude of the result."""
+    tol = TOL[name] if tol is None else tol
+    mag = max(1.0, float(np.abs(np64(ref)).max()))
+    err = max_abs(gpu, ref)
+    assert err <= tol * mag, (f"{name}: max|gpu-oracle| = {err:.3e} > {tol:.1e} * "
+                              f"max(1, max|ref| = {mag:.3e}) {ctx}")
+    return err
+
+
 def gpu_available():
     return torch.cuda.is_available()

@@ -6,7 +6,7 @@ import torch
 
 import oracle
 from tiled_attention_20_b200 import inputs
-from tests.parity import assert_close, np64
+from tests.parity import assert_close, assert_close_scaled, np64
 
 pytestmark = pytest.mark.gpu
 
@@ -28,13 +28,15 @@ def _run(B, H, N, d, causal, seed=0, dist="normal", grad_dtype=torch.bfloat16, s
     return (q, k, v, dO), (o, lse), (dq, dk, dv)
 
 
-def _check(B, H, N, d, causal, seed=0, dist="normal", grad_dtype=torch.bfloat16, scale=None):
+def _check(B, H, N, d, causal, seed=0, dist="normal", grad_dtype=torch.bfloat16, scale=None,
+           scaled_tol=False):
     (q, k, v, dO), (o, lse), (dq, dk, dv) = _run(B, H, N, d, causal, seed, dist, grad_dtype, scale)
     dq_r, dk_r, dv_r, _, _ = oracle.bwd(q, k, v, dO, scale=scale, causal=causal)
     ctx = f"B={B} H={H} N={N} d={d} causal={causal}"
-    e = {"dq": assert_close("dq", dq, dq_r, ctx=ctx),
-         "dk": assert_close("dk", dk, dk_r, ctx=ctx),
-         "dv": assert_close("dv", dv, dv_r, ctx=ctx)}
+    cmp = assert_close_scaled if scaled_tol else assert_close
+    e = {"dq": cmp("dq", dq, dq_r, ctx=ctx),
+         "dk": cmp("dk", dk, dk_r, ctx=ctx),
+         "dv": cmp("dv", dv, dv_r, ctx=ctx)}
     return e
 
 
@@ -66,15 +68,18 @@ def test_fp32_gradients(d):
 
 def test_scale_argument():
     """Non-default scales.  A larger scale sharpens the softmax and grows the
-    gradients, so the bf16 rounding of the outputs alone can exceed the
-    absolute bound; the check is made on fp32 gradient outputs."""
-    _check(1, 2, 257, 64, True, seed=11, scale=0.3, grad_dtype=torch.float32)
-    _check(1, 2, 257, 128, False, seed=12, scale=0.05, grad_dtype=torch.float32)
+    gradients (max|dQ| about 5.7 here), and bf16 operand rounding is relative,
+    so the bound is scaled by the magnitude of the result."""
+    _check(1, 2, 257, 64, True, seed=11, scale=0.3, scaled_tol=True)
+    _check(1, 2, 257, 64, True, seed=11, scale=0.3, grad_dtype=torch.float32, scaled_tol=True)
+    _check(1, 2, 257, 128, False, seed=12, scale=0.05)
 
 
 def test_long_context_distribution_small():
+    """Q, K ~ N(0, 3) with 1% of rows x8: logits in the hundreds and gradients
+    far from unit scale, so the bound is scaled by the result's magnitude."""
     for d in (64, 128):
-        _check(1, 2, 1100, d, True, seed=5, dist="long_context")
+        _check(1, 2, 1100, d, True, seed=5, dist="long_context", scaled_tol=True)
 
 
 @pytest.mark.parametrize("causal", [False, True])

@@ -19,18 +19,25 @@
 //      diagonal when causal) and keeps dK, dV accumulating in TMEM.
 //   3. fa_bwd_dq_convert: dQ = scale * accumulator, to the output dtype.
 //
-// Main kernel, 12 warps:
-//   warp 0      TMA producer: K_j, V_j once per unit; Q_i, dO_i, lse_i, D_i
-//               per Q block through a 3-slot ring.
+// Main kernel, 16 warps:
+//   warp 0      scheduler and TMA producer: takes the next work unit from a
+//               global atomic counter and publishes it to the other roles
+//               through a 4-entry ring in shared memory; loads K_j, V_j once
+//               per unit and Q_i, dO_i, lse_i, D_i per Q block (3-slot ring).
 //   warp 1      TMEM allocator and single-thread tcgen05.mma issuer.
-//   warps 4-7   "compute" warpgroup, one thread per key row: P^T from S^T
-//               and lse, dS^T = P^T (dP^T - D); P^T goes back to TMEM (A of
-//               dV += P^T dO), dS^T to shared memory (A of dK += dS^T Q and,
-//               read transposed, B of dQ^T = K^T dS^T); at the end of a unit
-//               it writes dK and dV.
-//   warps 8-11  dQ drain: one thread per head-dimension column; moves dQ^T
+//   warps 4-7   compute warpgroup 0, warps 8-11 compute warpgroup 1: they
+//               take alternate Q blocks (pipeline slot s = 0 / 1), one thread
+//               per key row: P^T from S^T and lse, dS^T = P^T (dP^T - D).
+//               P^T goes back to TMEM (A of dV += P^T dO), dS^T to shared
+//               memory (A of dK += dS^T Q and, read transposed, B of
+//               dQ^T = K^T dS^T).  At the end of a unit warpgroup 0 writes
+//               dV and warpgroup 1 writes dK.
+//   warps 12-15 dQ drain: one thread per head-dimension column; moves dQ^T
 //               from TMEM to shared memory and adds it into the fp32
 //               accumulator in global memory with bulk reduce-add copies.
+// Work units are ordered in groups of a few heads (so the dQ accumulator,
+// Q and dO of the heads in flight stay in L2), longest first (ascending K/V
+// block) within a group, and handed out dynamically.
 // TMEM columns: dV [0,D) dK [D,2D) S^T_s [2D+64s, +64) dP^T_s [2D+128+64s, +64)
 // for the two pipeline slots s; dQ^T of slot s overwrites dP^T_s once the
 // compute warps have read it, P^T_s (bf16 pairs) overwrites S^T_s.
@@ -44,12 +51,17 @@ inline int bwd_units(int B, int H, int N) { return B * H * ((N + 127) / 128); }
 inline size_t round256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
 
 // Workspace: dQ accumulator [BH][N][d] fp32, then lse*log2e and D, each
-// [BH][Npad] fp32 with Npad = N rounded up to 64.
+// [BH][Npad] fp32 with Npad = N rounded up to 64, then the scheduler's
+// work-unit counter.
 inline size_t bwd_npad(int N) { return (static_cast<size_t>(N) + 63) / 64 * 64; }
 inline size_t bwd_workspace_bytes(int B, int H, int N, int d) {
   const size_t bh = static_cast<size_t>(B) * H;
-  return round256(bh * N * d * 4) + 2 * round256(bh * bwd_npad(N) * 4);
+  return round256(bh * N * d * 4) + 2 * round256(bh * bwd_npad(N) * 4) + 256;
 }
+
+// Heads per scheduling group: the heads in flight keep their K, V, Q, dO and
+// dQ accumulator in L2.
+constexpr int kBwdGroupHeads = 8;
 
 struct BwdParams {
   void* dk;
@@ -57,6 +69,7 @@ struct BwdParams {
   float* dq_acc;
   const float* lse2;  // [BH][Npad]
   const float* dvec;  // [BH][Npad]
+  int* sched;         // work-unit counter, zero at launch
   int BH;
   int N;
   int Npad;
@@ -95,12 +108,19 @@ struct BwdLayout {
   static constexpr uint32_t kTdP = 2 * D + 128;  // + 64 s
 };
 
+constexpr int kUnitRing = 4;
+// Consumers of the unit ring, counted in arrivals: the MMA thread, the 8
+// compute warps and the 4 drain warps (one lane each).
+constexpr int kUnitConsumers = 1 + 8 + 4;
+
 struct BwdBarriers {
   uint64_t kv_full, kv_empty;
   uint64_t q_full[3], q_empty[3];
   uint64_t s_full[2], dp_full[2], p_ready[2], ds_ready[2], dq_full[2], dq_empty[2];
-  uint64_t acc_full;
+  uint64_t acc_full, acc_empty;
+  uint64_t unit_full[kUnitRing], unit_empty[kUnitRing];
   uint64_t mma_done;
+  int unit_id[kUnitRing];
   uint32_t tmem_base;
   int abort_flag;
 };
@@ -109,11 +129,18 @@ struct BwdUnit {
   int bh, j, i0, n;  // head, K/V block, first Q block, number of Q blocks
 };
 
+// Unit w -> (head, K/V block): groups of kBwdGroupHeads heads, K/V blocks in
+// ascending order within a group (the longest causal units first), heads
+// innermost.
 template <bool CAUSAL>
 __device__ __forceinline__ BwdUnit bwd_decode(const BwdParams& p, int w) {
   BwdUnit u;
-  u.j = w / p.BH;  // causal: ascending j = longest first
-  u.bh = w - u.j * p.BH;
+  const int per_group = kBwdGroupHeads * p.nkv;
+  const int g = w / per_group;
+  const int r = w - g * per_group;
+  const int heads = min(kBwdGroupHeads, p.BH - g * kBwdGroupHeads);
+  u.j = r / heads;
+  u.bh = g * kBwdGroupHeads + (r - u.j * heads);
   u.i0 = CAUSAL ? 2 * u.j : 0;
   u.n = p.nq - u.i0;
   return u;
@@ -134,6 +161,28 @@ __device__ __forceinline__ bool bwait_warp(uint64_t* bar, uint32_t parity, BwdBa
   ok = __all_sync(0xffffffffu, ok);
   if (!ok) *(volatile int*)&b->abort_flag = 1;
   return ok;
+}
+
+// Next unit from the ring for a consumer warp (all 32 lanes call; lane 0
+// releases the entry).  Returns -1 when the schedule is exhausted, -2 on abort.
+__device__ __forceinline__ int next_unit_warp(BwdBarriers* b, int& rc, int* status) {
+  const int slot = rc % kUnitRing;
+  if (!bwait_warp(&b->unit_full[slot], (rc / kUnitRing) & 1, b, status)) return -2;
+  const int w = *(volatile int*)&b->unit_id[slot];
+  __syncwarp();
+  if (lane_id() == 0) mbar_arrive(&b->unit_empty[slot]);
+  ++rc;
+  return w;
+}
+
+// The same for the single MMA thread.
+__device__ __forceinline__ int next_unit_one(BwdBarriers* b, int& rc, int* status) {
+  const int slot = rc % kUnitRing;
+  if (!bwait1(&b->unit_full[slot], (rc / kUnitRing) & 1, b, status)) return -2;
+  const int w = *(volatile int*)&b->unit_id[slot];
+  mbar_arrive(&b->unit_empty[slot]);
+  ++rc;
+  return w;
 }
 
 __device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t bytes,
@@ -193,7 +242,16 @@ __device__ void bwd_producer(const CUtensorMap* tm_q, const CUtensorMap* tm_k,
                              int& kvc) {
   using L = BwdLayout<D>;
   constexpr int QS = L::kQStages;
-  for (int w = blockIdx.x; w < p.n_units; w += gridDim.x) {
+  for (int uc = 0;; ++uc) {
+    // Take the next unit and publish it to the other roles.
+    const int slot = uc % kUnitRing;
+    if (uc >= kUnitRing && !bwait1(&b->unit_empty[slot], ((uc / kUnitRing) - 1) & 1, b, p.status))
+      return;
+    int w = atomicAdd(p.sched, 1);
+    if (w >= p.n_units) w = -1;
+    *(volatile int*)&b->unit_id[slot] = w;
+    mbar_arrive(&b->unit_full[slot]);
+    if (w < 0) return;
     const BwdUnit u = bwd_decode<CAUSAL>(p, w);
     // Prefetch the first Q blocks of this unit before waiting for the K/V
     // buffers, which the previous unit may still be using.
@@ -272,8 +330,10 @@ __device__ void bwd_mma(const BwdParams& p, uint8_t* smem, BwdBarriers* b, uint3
   const uint32_t sb = smem_u32(smem);
   int g = 0;      // global Q-block iteration counter (pipeline slot = g % 2)
   int qbase = 0;  // Q-ring uses before this unit
-  int uc = 0;     // units processed
-  for (int w = blockIdx.x; w < p.n_units; w += gridDim.x, ++uc) {
+  int rc = 0;     // unit-ring reads
+  for (int uc = 0;; ++uc) {
+    const int w = next_unit_one(b, rc, p.status);
+    if (w < 0) return;
     const BwdUnit u = bwd_decode<CAUSAL>(p, w);
     if (!bwait1(&b->kv_full, uc & 1, b, p.status)) return;
     tc_fence_after();
@@ -293,6 +353,10 @@ __device__ void bwd_mma(const BwdParams& p, uint8_t* smem, BwdBarriers* b, uint3
     };
     auto grads = [&](int it) -> bool {
       const int gg = g + it, s = gg & 1, qi = qbase + it, qs = qi % QS;
+      if (it == 0 && uc > 0) {  // the previous unit's dK, dV have been written out
+        if (!bwait1(&b->acc_empty, (uc - 1) & 1, b, p.status)) return false;
+        tc_fence_after();
+      }
       if (!bwait1(&b->p_ready[s], (gg >> 1) & 1, b, p.status)) return false;
       tc_fence_after();
       M::dv(tmem + L::kTdV, tmem + L::kTS + 64 * s, sb + L::kDO + qs * L::kQBytes, it > 0);
@@ -317,113 +381,115 @@ __device__ void bwd_mma(const BwdParams& p, uint8_t* smem, BwdBarriers* b, uint3
   }
 }
 
-// ---------------------------------------------------------------- compute warpgroup
+// ---------------------------------------------------------------- compute warpgroups
 template <int D, bool CAUSAL>
-__device__ void bwd_compute(const BwdParams& p, uint8_t* smem, BwdBarriers* b, uint32_t tmem) {
+__device__ void bwd_compute(const BwdParams& p, uint8_t* smem, BwdBarriers* b, uint32_t tmem,
+                            int s) {
   using L = BwdLayout<D>;
   constexpr int QS = L::kQStages;
-  const int t = threadIdx.x - 128;  // key row within the K/V block == TMEM lane
+  const int t = (threadIdx.x - 128) & 127;  // key row within the K/V block == TMEM lane
   const uint32_t lane_base = static_cast<uint32_t>(t & ~31) << 16;
   const float sl2 = p.scale_log2;
-  int g = 0, qbase = 0, uc = 0;
-  for (int w = blockIdx.x; w < p.n_units; w += gridDim.x, ++uc) {
+  const uint32_t tS = tmem + lane_base + L::kTS + 64 * s;
+  const uint32_t tdP = tmem + lane_base + L::kTdP + 64 * s;
+  uint8_t* ds_row = smem + L::kDs + s * L::kDsBytes + t * 128;
+  int g = 0, qbase = 0, rc = 0;
+  for (int uc = 0;; ++uc) {
+    const int w = next_unit_warp(b, rc, p.status);
+    if (w < 0) return;
     const BwdUnit u = bwd_decode<CAUSAL>(p, w);
     const int key = u.j * 128 + t;
     for (int it = 0; it < u.n; ++it) {
-      const int gg = g + it, s = gg & 1, qs = (qbase + it) % QS;
+      const int gg = g + it;
+      if ((gg & 1) != s) continue;
+      const int qs = (qbase + it) % QS;
       const int q0 = (u.i0 + it) * 64;
       if (!bwait_warp(&b->s_full[s], (gg >> 1) & 1, b, p.status)) return;
-      tc_fence_after();
-      float pr[64];
-      {
-        uint32_t r[64];
-        tmem_ld_x64(tmem + lane_base + L::kTS + 64 * s, r);
-        const float4* lse4 = reinterpret_cast<const float4*>(smem + L::kLse + qs * 256);
-#pragma unroll
-        for (int c4 = 0; c4 < 16; ++c4) {
-          const float4 l4 = lse4[c4];
-          pr[4 * c4 + 0] = ex2_approx(fmaf(__uint_as_float(r[4 * c4 + 0]), sl2, -l4.x));
-          pr[4 * c4 + 1] = ex2_approx(fmaf(__uint_as_float(r[4 * c4 + 1]), sl2, -l4.y));
-          pr[4 * c4 + 2] = ex2_approx(fmaf(__uint_as_float(r[4 * c4 + 2]), sl2, -l4.z));
-          pr[4 * c4 + 3] = ex2_approx(fmaf(__uint_as_float(r[4 * c4 + 3]), sl2, -l4.w));
-        }
-      }
-      if (CAUSAL && q0 < u.j * 128 + 127) {
-#pragma unroll
-        for (int c = 0; c < 64; ++c) pr[c] = (key <= q0 + c) ? pr[c] : 0.f;
-      }
-      {
-        uint32_t pk[32];
-#pragma unroll
-        for (int c = 0; c < 32; ++c) pk[c] = pack_bf16x2(pr[2 * c], pr[2 * c + 1]);
-        tmem_st_x32(tmem + lane_base + L::kTS + 64 * s, pk);
-        tmem_st_wait();
-      }
-      tc_fence_before();
-      mbar_arrive(&b->p_ready[s]);
       if (!bwait_warp(&b->dp_full[s], (gg >> 1) & 1, b, p.status)) return;
       tc_fence_after();
-      {
-        uint32_t r[64];
-        tmem_ld_x64(tmem + lane_base + L::kTdP + 64 * s, r);
-        const float4* dv4 = reinterpret_cast<const float4*>(smem + L::kDv + qs * 256);
-        uint8_t* ds_row = smem + L::kDs + s * L::kDsBytes + t * 128;
+      const float4* lse4 = reinterpret_cast<const float4*>(smem + L::kLse + qs * 256);
+      const float4* dv4 = reinterpret_cast<const float4*>(smem + L::kDv + qs * 256);
+      const bool diag = CAUSAL && q0 < u.j * 128 + 127;
 #pragma unroll
-        for (int piece = 0; piece < 8; ++piece) {  // 8 queries = 16 bytes per piece
-          const float4 da = dv4[2 * piece], db = dv4[2 * piece + 1];
-          const int c = piece * 8;
+      for (int h = 0; h < 2; ++h) {
+        uint32_t rs[32], rp[32];
+        tmem_ld_x32(tS + 32 * h, rs);
+        tmem_ld_x32(tdP + 32 * h, rp);
+        float pr[32];
+#pragma unroll
+        for (int c4 = 0; c4 < 8; ++c4) {
+          const float4 l4 = lse4[8 * h + c4];
+          pr[4 * c4 + 0] = ex2_approx(fmaf(__uint_as_float(rs[4 * c4 + 0]), sl2, -l4.x));
+          pr[4 * c4 + 1] = ex2_approx(fmaf(__uint_as_float(rs[4 * c4 + 1]), sl2, -l4.y));
+          pr[4 * c4 + 2] = ex2_approx(fmaf(__uint_as_float(rs[4 * c4 + 2]), sl2, -l4.z));
+          pr[4 * c4 + 3] = ex2_approx(fmaf(__uint_as_float(rs[4 * c4 + 3]), sl2, -l4.w));
+        }
+        if (diag) {
+#pragma unroll
+          for (int c = 0; c < 32; ++c) pr[c] = (key <= q0 + 32 * h + c) ? pr[c] : 0.f;
+        }
+        uint32_t pk[16];
+#pragma unroll
+        for (int c = 0; c < 16; ++c) pk[c] = pack_bf16x2(pr[2 * c], pr[2 * c + 1]);
+        tmem_st_x16(tS + 16 * h, pk);
+#pragma unroll
+        for (int piece = 0; piece < 4; ++piece) {  // 8 queries = 16 bytes per piece
+          const float4 da = dv4[8 * h + 2 * piece], db = dv4[8 * h + 2 * piece + 1];
           const float d8[8] = {da.x, da.y, da.z, da.w, db.x, db.y, db.z, db.w};
           uint32_t w4[4];
 #pragma unroll
           for (int e = 0; e < 4; ++e) {
-            const float ds0 = pr[c + 2 * e] * (__uint_as_float(r[c + 2 * e]) - d8[2 * e]);
-            const float ds1 = pr[c + 2 * e + 1] * (__uint_as_float(r[c + 2 * e + 1]) - d8[2 * e + 1]);
+            const int c = piece * 8 + 2 * e;
+            const float ds0 = pr[c] * (__uint_as_float(rp[c]) - d8[2 * e]);
+            const float ds1 = pr[c + 1] * (__uint_as_float(rp[c + 1]) - d8[2 * e + 1]);
             w4[e] = pack_bf16x2(ds0, ds1);
           }
           // 128-byte swizzle: 16-byte piece index XOR (row mod 8).
-          *reinterpret_cast<uint4*>(ds_row + ((piece ^ (t & 7)) << 4)) =
+          const int pc = 4 * h + piece;
+          *reinterpret_cast<uint4*>(ds_row + ((pc ^ (t & 7)) << 4)) =
               make_uint4(w4[0], w4[1], w4[2], w4[3]);
         }
       }
-      fence_proxy_async_smem();
+      tmem_st_wait();
       tc_fence_before();
+      mbar_arrive(&b->p_ready[s]);
+      fence_proxy_async_smem();
       mbar_arrive(&b->ds_ready[s]);
     }
-    // Unit epilogue: dV and scale * dK for this thread's key row.
+    // Unit epilogue: warpgroup 0 writes dV, warpgroup 1 writes scale * dK.
     if (!bwait_warp(&b->acc_full, uc & 1, b, p.status)) return;
     tc_fence_after();
     const bool valid = key < p.N;
     const size_t row = static_cast<size_t>(u.bh) * p.N + key;
+    const uint32_t col = s ? L::kTdK : L::kTdV;
+    const float mul = s ? p.scale : 1.f;
+    void* out = s ? p.dk : p.dv;
 #pragma unroll
-    for (int which = 0; which < 2; ++which) {
-      const uint32_t col = which ? L::kTdK : L::kTdV;
-      const float mul = which ? p.scale : 1.f;
-      void* out = which ? p.dk : p.dv;
+    for (int c0 = 0; c0 < D; c0 += 32) {
+      uint32_t r[32];
+      tmem_ld_x32(tmem + lane_base + col + c0, r);
+      if (valid) {
+        if (p.grad_f32) {
+          float4* dst = reinterpret_cast<float4*>(static_cast<float*>(out) + row * D + c0);
 #pragma unroll
-      for (int c0 = 0; c0 < D; c0 += 32) {
-        uint32_t r[32];
-        tmem_ld_x32(tmem + lane_base + col + c0, r);
-        if (valid) {
-          if (p.grad_f32) {
-            float4* dst = reinterpret_cast<float4*>(static_cast<float*>(out) + row * D + c0);
+          for (int v = 0; v < 8; ++v)
+            dst[v] = make_float4(__uint_as_float(r[4 * v]) * mul, __uint_as_float(r[4 * v + 1]) * mul,
+                                 __uint_as_float(r[4 * v + 2]) * mul,
+                                 __uint_as_float(r[4 * v + 3]) * mul);
+        } else {
+          uint4* dst = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(out) + row * D + c0);
 #pragma unroll
-            for (int v = 0; v < 8; ++v)
-              dst[v] = make_float4(__uint_as_float(r[4 * v]) * mul, __uint_as_float(r[4 * v + 1]) * mul,
-                                   __uint_as_float(r[4 * v + 2]) * mul,
-                                   __uint_as_float(r[4 * v + 3]) * mul);
-          } else {
-            uint4* dst = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(out) + row * D + c0);
-#pragma unroll
-            for (int v = 0; v < 4; ++v)
-              dst[v] = make_uint4(
-                  pack_bf16x2(__uint_as_float(r[8 * v + 0]) * mul, __uint_as_float(r[8 * v + 1]) * mul),
-                  pack_bf16x2(__uint_as_float(r[8 * v + 2]) * mul, __uint_as_float(r[8 * v + 3]) * mul),
-                  pack_bf16x2(__uint_as_float(r[8 * v + 4]) * mul, __uint_as_float(r[8 * v + 5]) * mul),
-                  pack_bf16x2(__uint_as_float(r[8 * v + 6]) * mul, __uint_as_float(r[8 * v + 7]) * mul));
-          }
+          for (int v = 0; v < 4; ++v)
+            dst[v] = make_uint4(
+                pack_bf16x2(__uint_as_float(r[8 * v + 0]) * mul, __uint_as_float(r[8 * v + 1]) * mul),
+                pack_bf16x2(__uint_as_float(r[8 * v + 2]) * mul, __uint_as_float(r[8 * v + 3]) * mul),
+                pack_bf16x2(__uint_as_float(r[8 * v + 4]) * mul, __uint_as_float(r[8 * v + 5]) * mul),
+                pack_bf16x2(__uint_as_float(r[8 * v + 6]) * mul, __uint_as_float(r[8 * v + 7]) * mul));
         }
       }
     }
+    tc_fence_before();
+    mbar_arrive(&b->acc_empty);
     g += u.n;
     qbase += u.n;
   }
@@ -433,7 +499,7 @@ __device__ void bwd_compute(const BwdParams& p, uint8_t* smem, BwdBarriers* b, u
 template <int D, bool CAUSAL>
 __device__ void bwd_drain(const BwdParams& p, uint8_t* smem, BwdBarriers* b, uint32_t tmem) {
   using L = BwdLayout<D>;
-  const int t = threadIdx.x - 256;
+  const int t = threadIdx.x - 384;
   const int quarter = t >> 5, ln = t & 31;
   const uint32_t lane_base = static_cast<uint32_t>(quarter * 32) << 16;
   // M = D accumulator layout: D = 128 fills all 128 lanes (lane = column of
@@ -442,13 +508,18 @@ __device__ void bwd_drain(const BwdParams& p, uint8_t* smem, BwdBarriers* b, uin
   const int dcol = (D == 128) ? t : (quarter * 16 + ln);
   const bool issuer = (t == 0);
   float* stage = reinterpret_cast<float*>(smem + L::kStage);
-  int g = 0;
-  for (int w = blockIdx.x; w < p.n_units; w += gridDim.x) {
+  int g = 0, rc = 0;
+  for (;;) {
+    const int w = next_unit_warp(b, rc, p.status);
+    if (w < 0) break;
     const BwdUnit u = bwd_decode<CAUSAL>(p, w);
     for (int it = 0; it < u.n; ++it, ++g) {
       const int s = g & 1;
       const int q0 = (u.i0 + it) * 64;
-      if (!bwait_warp(&b->dq_full[s], (g >> 1) & 1, b, p.status)) return;
+      if (!bwait_warp(&b->dq_full[s], (g >> 1) & 1, b, p.status)) {
+        if (issuer) bulk_wait0();
+        return;
+      }
       tc_fence_after();
       uint32_t r[64];
       tmem_ld_x64(tmem + lane_base + L::kTdP + 64 * s, r);
@@ -482,7 +553,7 @@ __device__ void bwd_drain(const BwdParams& p, uint8_t* smem, BwdBarriers* b, uin
 
 // ---------------------------------------------------------------- kernels
 template <int D, bool CAUSAL>
-__global__ void __launch_bounds__(384, 1)
+__global__ void __launch_bounds__(512, 1)
     fa_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                   const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
                   const BwdParams p) {
@@ -508,6 +579,11 @@ __global__ void __launch_bounds__(384, 1)
       mbar_init(&b->dq_empty[i], 128);
     }
     mbar_init(&b->acc_full, 1);
+    mbar_init(&b->acc_empty, 256);
+    for (int i = 0; i < kUnitRing; ++i) {
+      mbar_init(&b->unit_full[i], 1);
+      mbar_init(&b->unit_empty[i], kUnitConsumers);
+    }
     mbar_init(&b->mma_done, 1);
     b->abort_flag = 0;
     fence_barrier_init();
@@ -547,9 +623,9 @@ __global__ void __launch_bounds__(384, 1)
       mbar_wait(&b->mma_done, 0, p.status);
     }
     __syncwarp();
-  } else if (warp >= 4 && warp < 8) {
-    bwd_compute<D, CAUSAL>(p, smem, b, tmem);
-  } else if (warp >= 8) {
+  } else if (warp >= 4 && warp < 12) {
+    bwd_compute<D, CAUSAL>(p, smem, b, tmem, (warp - 4) >> 2);
+  } else if (warp >= 12) {
     bwd_drain<D, CAUSAL>(p, smem, b, tmem);
   }
   tc_fence_before();
@@ -559,13 +635,14 @@ __global__ void __launch_bounds__(384, 1)
 }
 
 // D_i = rowsum(dO * O); lse2 = lse * log2(e) (+inf and D = 0 on rows N..Npad);
-// zero the dQ accumulator.  One thread per 8 consecutive elements of a row.
+// zero the dQ accumulator and the work-unit counter.  One thread per 8 consecutive elements of a row.
 template <int D>
 __global__ void __launch_bounds__(256)
     fa_bwd_prep(const __nv_bfloat16* __restrict__ o, const __nv_bfloat16* __restrict__ dO,
                 const float* __restrict__ lse, float* __restrict__ lse2, float* __restrict__ dvec,
-                float* __restrict__ dq_acc, int BH, int N, int Npad) {
+                float* __restrict__ dq_acc, int* __restrict__ sched, int BH, int N, int Npad) {
   constexpr int TPR = D / 8;  // threads per row
+  if (blockIdx.x == 0 && threadIdx.x == 0) *sched = 0;
   const long long gid = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x;
   const long long row = gid / TPR;  // over BH * Npad
   const int part = static_cast<int>(gid % TPR);
@@ -617,101 +694,6 @@ __global__ void __launch_bounds__(256)
         make_uint4(pack_bf16x2(a.x * scale, a.y * scale), pack_bf16x2(a.z * scale, a.w * scale),
                    pack_bf16x2(c.x * scale, c.y * scale), pack_bf16x2(c.z * scale, c.w * scale));
   }
-}
-
-typedef CUresult (*EncodeTiledFnT)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
-                                   const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
-                                   const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
-                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
-
-inline int bwd_tmap(EncodeTiledFnT enc, CUtensorMap* m, const void* base, int BH, int N, int d,
-                    int box_rows) {
-  cuuint64_t dims[3] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(N),
-                        static_cast<cuuint64_t>(BH)};
-  cuuint64_t strides[2] = {static_cast<cuuint64_t>(d) * 2, static_cast<cuuint64_t>(N) * d * 2};
-  cuuint32_t box[3] = {64, static_cast<cuuint32_t>(box_rows), 1};
-  cuuint32_t estr[3] = {1, 1, 1};
-  CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides,
-                   box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-  return r == CUDA_SUCCESS ? 0 : -6;
-}
-
-template <int D, bool CAUSAL>
-inline int launch_bwd_t(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
-                        const CUtensorMap& tdo, const BwdParams& p, int ctas,
-                        cudaStream_t stream) {
-  auto kern = fa_bwd_kernel<D, CAUSAL>;
-  const int smem = BwdLayout<D>::kSmemBytes;
-  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
-    return -6;
-  kern<<<ctas, 384, smem, stream>>>(tq, tk, tv, tdo, p);
-  return cudaPeekAtLastError() == cudaSuccess ? 0 : -6;
-}
-
-inline int launch_bwd(const void* q, const void* k, const void* v, const void* o, const void* dO,
-                      const float* lse, void* dq, void* dk, void* dv, int B, int H, int N, int d,
-                      float scale, bool causal, void* workspace, int grad_dtype, int sms,
-                      int* status, cudaStream_t stream, EncodeTiledFnT enc) {
-  const int BH = B * H;
-  const size_t npad = bwd_npad(N);
-  uint8_t* ws = static_cast<uint8_t*>(workspace);
-  float* dq_acc = reinterpret_cast<float*>(ws);
-  float* lse2 = reinterpret_cast<float*>(ws + round256(static_cast<size_t>(BH) * N * d * 4));
-  float* dvec = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(lse2) +
-                                         round256(static_cast<size_t>(BH) * npad * 4));
-  // 1. preprocess
-  {
-    const long long threads = static_cast<long long>(BH) * npad * (d / 8);
-    const int blocks = static_cast<int>((threads + 255) / 256);
-    if (d == 64)
-      fa_bwd_prep<64><<<blocks, 256, 0, stream>>>(static_cast<const __nv_bfloat16*>(o),
-                                                   static_cast<const __nv_bfloat16*>(dO), lse, lse2,
-                                                   dvec, dq_acc, BH, N, static_cast<int>(npad));
-    else
-      fa_bwd_prep<128><<<blocks, 256, 0, stream>>>(static_cast<const __nv_bfloat16*>(o),
-                                                    static_cast<const __nv_bfloat16*>(dO), lse, lse2,
-                                                    dvec, dq_acc, BH, N, static_cast<int>(npad));
-    if (cudaPeekAtLastError() != cudaSuccess) return -6;
-  }
-  // 2. main kernel
-  CUtensorMap tq, tk, tv, tdo;
-  if (bwd_tmap(enc, &tq, q, BH, N, d, 64) || bwd_tmap(enc, &tdo, dO, BH, N, d, 64) ||
-      bwd_tmap(enc, &tk, k, BH, N, d, 128) || bwd_tmap(enc, &tv, v, BH, N, d, 128))
-    return -6;
-  BwdParams p;
-  p.dk = dk;
-  p.dv = dv;
-  p.dq_acc = dq_acc;
-  p.lse2 = lse2;
-  p.dvec = dvec;
-  p.BH = BH;
-  p.N = N;
-  p.Npad = static_cast<int>(npad);
-  p.nq = (N + 63) / 64;
-  p.nkv = (N + 127) / 128;
-  p.n_units = BH * p.nkv;
-  p.scale_log2 = scale * 1.4426950408889634f;
-  p.scale = scale;
-  p.grad_f32 = grad_dtype;
-  p.status = status;
-  const int ctas = p.n_units < sms ? p.n_units : sms;
-  int rc;
-  if (d == 64)
-    rc = causal ? launch_bwd_t<64, true>(tq, tk, tv, tdo, p, ctas, stream)
-                : launch_bwd_t<64, false>(tq, tk, tv, tdo, p, ctas, stream);
-  else
-    rc = causal ? launch_bwd_t<128, true>(tq, tk, tv, tdo, p, ctas, stream)
-                : launch_bwd_t<128, false>(tq, tk, tv, tdo, p, ctas, stream);
-  if (rc) return rc;
-  // 3. dQ conversion
-  {
-    const long long n8 = static_cast<long long>(BH) * N * d / 8;
-    const int blocks = static_cast<int>((n8 + 255) / 256);
-    fa_bwd_dq_convert<<<blocks, 256, 0, stream>>>(dq_acc, dq, n8, scale, grad_dtype);
-    if (cudaPeekAtLastError() != cudaSuccess) return -6;
-  }
-  return 0;
 }
 
 }  // namespace fa

@@ -6,6 +6,7 @@
 #include <cstdint>
 #include <cstring>
 #include <mutex>
+#include <vector>
 
 #include <cuda.h>
 #include <cuda_runtime.h>
@@ -37,6 +38,58 @@ typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t,
                                   const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
 EncodeTiledFn g_encode = nullptr;
+
+// ---------------------------------------------------------------- tracing
+// Opt-in per-kernel timing: while enabled, every launch is bracketed by a
+// pair of CUDA events on its stream.
+enum { kKernFwd = 0, kKernBwdPrep = 1, kKernBwd = 2, kKernBwdConvert = 3, kNumKernels = 4 };
+const char* const kKernelNames[kNumKernels] = {"fa_fwd_kernel", "fa_bwd_prep", "fa_bwd_kernel",
+                                               "fa_bwd_dq_convert"};
+struct TraceRec {
+  int kernel;
+  int device;
+  cudaEvent_t start, stop;
+};
+std::mutex g_trace_mu;
+bool g_trace_on = false;
+std::vector<TraceRec> g_trace;
+std::vector<cudaEvent_t> g_event_pool[kMaxDevices];
+size_t g_event_used[kMaxDevices];
+
+cudaEvent_t trace_event(int dev) {
+  if (g_event_used[dev] == g_event_pool[dev].size()) {
+    cudaEvent_t e;
+    if (cudaEventCreate(&e) != cudaSuccess) return nullptr;
+    g_event_pool[dev].push_back(e);
+  }
+  return g_event_pool[dev][g_event_used[dev]++];
+}
+
+// Brackets one launch when tracing is on.
+class LaunchTrace {
+ public:
+  LaunchTrace(int kernel, cudaStream_t s) : stream_(s) {
+    std::lock_guard<std::mutex> lock(g_trace_mu);
+    if (!g_trace_on) return;
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return;
+    rec_.kernel = kernel;
+    rec_.device = dev;
+    rec_.start = trace_event(dev);
+    rec_.stop = trace_event(dev);
+    if (rec_.start && rec_.stop && cudaEventRecord(rec_.start, s) == cudaSuccess) active_ = true;
+  }
+  ~LaunchTrace() {
+    if (!active_) return;
+    std::lock_guard<std::mutex> lock(g_trace_mu);
+    if (cudaEventRecord(rec_.stop, stream_) == cudaSuccess) g_trace.push_back(rec_);
+  }
+
+ private:
+  cudaStream_t stream_;
+  TraceRec rec_{};
+  bool active_ = false;
+};
 
 // Fills *info for the current device (once per device).
 int device_info(DeviceInfo** info) {
@@ -82,22 +135,7 @@ int check_scale(float scale) {
   return FA_OK;
 }
 
-// 3-D view [B*H][N][d] of a bf16 tensor, boxes of 128 rows x 64 columns with
-// 128-byte swizzle.  Rows past N read as zero (the third dimension keeps
-// one head's ragged tail from reading the next head's rows).
-int make_tmap(CUtensorMap* m, const void* base, int BH, int N, int d) {
-  cuuint64_t dims[3] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(N),
-                        static_cast<cuuint64_t>(BH)};
-  cuuint64_t strides[2] = {static_cast<cuuint64_t>(d) * 2,
-                           static_cast<cuuint64_t>(N) * d * 2};
-  cuuint32_t box[3] = {64, 128, 1};
-  cuuint32_t estr[3] = {1, 1, 1};
-  CUresult r = g_encode(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims,
-                        strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
-                        CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-                        CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-  return r == CUDA_SUCCESS ? FA_OK : FA_ERR_LAUNCH;
-}
+int make_tmap_rows(CUtensorMap* m, const void* base, int BH, int N, int d, int box_rows);
 
 int fwd_units(int B, int H, int N) { return B * H * ((N + 255) / 256); }
 
@@ -108,8 +146,109 @@ int launch_fwd(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& 
   const int smem = fa::FwdLayout<D>::kSmemBytes;
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
     return FA_ERR_LAUNCH;
+  LaunchTrace trace(kKernFwd, stream);
   kern<<<ctas, 384, smem, stream>>>(tq, tk, tv, p);
   return cudaPeekAtLastError() == cudaSuccess ? FA_OK : FA_ERR_LAUNCH;
+}
+
+// ---------------------------------------------------------------- backward launches
+// 3-D view [B*H][N][d] of a bf16 tensor, boxes of `box_rows` rows x 64
+// columns with 128-byte swizzle.  Rows past N read as zero (the third
+// dimension keeps one head's ragged tail from reading the next head's rows).
+int make_tmap_rows(CUtensorMap* m, const void* base, int BH, int N, int d, int box_rows) {
+  cuuint64_t dims[3] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(N),
+                        static_cast<cuuint64_t>(BH)};
+  cuuint64_t strides[2] = {static_cast<cuuint64_t>(d) * 2, static_cast<cuuint64_t>(N) * d * 2};
+  cuuint32_t box[3] = {64, static_cast<cuuint32_t>(box_rows), 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = g_encode(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims,
+                        strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                        CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                        CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? FA_OK : FA_ERR_LAUNCH;
+}
+
+template <int D, bool CAUSAL>
+int launch_bwd_main(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
+                    const CUtensorMap& tdo, const fa::BwdParams& p, int ctas,
+                    cudaStream_t stream) {
+  auto kern = fa::fa_bwd_kernel<D, CAUSAL>;
+  const int smem = fa::BwdLayout<D>::kSmemBytes;
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
+    return FA_ERR_LAUNCH;
+  LaunchTrace trace(kKernBwd, stream);
+  kern<<<ctas, 512, smem, stream>>>(tq, tk, tv, tdo, p);
+  return cudaPeekAtLastError() == cudaSuccess ? FA_OK : FA_ERR_LAUNCH;
+}
+
+int launch_bwd(const void* q, const void* k, const void* v, const void* o, const void* dO,
+               const float* lse, void* dq, void* dk, void* dv, int B, int H, int N, int d,
+               float scale, bool causal, void* workspace, int grad_dtype, int sms, int* status,
+               cudaStream_t stream) {
+  const int BH = B * H;
+  const size_t npad = fa::bwd_npad(N);
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  float* dq_acc = reinterpret_cast<float*>(ws);
+  float* lse2 = reinterpret_cast<float*>(ws + fa::round256(static_cast<size_t>(BH) * N * d * 4));
+  float* dvec = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(lse2) +
+                                         fa::round256(static_cast<size_t>(BH) * npad * 4));
+  int* sched = reinterpret_cast<int*>(reinterpret_cast<uint8_t*>(dvec) +
+                                      fa::round256(static_cast<size_t>(BH) * npad * 4));
+  CUtensorMap tq, tk, tv, tdo;
+  if (make_tmap_rows(&tq, q, BH, N, d, 64) != FA_OK || make_tmap_rows(&tdo, dO, BH, N, d, 64) != FA_OK ||
+      make_tmap_rows(&tk, k, BH, N, d, 128) != FA_OK || make_tmap_rows(&tv, v, BH, N, d, 128) != FA_OK)
+    return FA_ERR_LAUNCH;
+  // 1. D, lse * log2(e), zeroed dQ accumulator
+  {
+    const long long threads = static_cast<long long>(BH) * npad * (d / 8);
+    const int blocks = static_cast<int>((threads + 255) / 256);
+    LaunchTrace trace(kKernBwdPrep, stream);
+    if (d == 64)
+      fa::fa_bwd_prep<64><<<blocks, 256, 0, stream>>>(
+          static_cast<const __nv_bfloat16*>(o), static_cast<const __nv_bfloat16*>(dO), lse, lse2,
+          dvec, dq_acc, sched, BH, N, static_cast<int>(npad));
+    else
+      fa::fa_bwd_prep<128><<<blocks, 256, 0, stream>>>(
+          static_cast<const __nv_bfloat16*>(o), static_cast<const __nv_bfloat16*>(dO), lse, lse2,
+          dvec, dq_acc, sched, BH, N, static_cast<int>(npad));
+    if (cudaPeekAtLastError() != cudaSuccess) return FA_ERR_LAUNCH;
+  }
+  // 2. tensor-core main kernel
+  fa::BwdParams p;
+  p.dk = dk;
+  p.dv = dv;
+  p.dq_acc = dq_acc;
+  p.lse2 = lse2;
+  p.dvec = dvec;
+  p.sched = sched;
+  p.BH = BH;
+  p.N = N;
+  p.Npad = static_cast<int>(npad);
+  p.nq = (N + 63) / 64;
+  p.nkv = (N + 127) / 128;
+  p.n_units = BH * p.nkv;
+  p.scale_log2 = scale * 1.4426950408889634f;
+  p.scale = scale;
+  p.grad_f32 = grad_dtype;
+  p.status = status;
+  const int ctas = p.n_units < sms ? p.n_units : sms;
+  int rc;
+  if (d == 64)
+    rc = causal ? launch_bwd_main<64, true>(tq, tk, tv, tdo, p, ctas, stream)
+                : launch_bwd_main<64, false>(tq, tk, tv, tdo, p, ctas, stream);
+  else
+    rc = causal ? launch_bwd_main<128, true>(tq, tk, tv, tdo, p, ctas, stream)
+                : launch_bwd_main<128, false>(tq, tk, tv, tdo, p, ctas, stream);
+  if (rc != FA_OK) return rc;
+  // 3. dQ = scale * accumulator
+  {
+    const long long n8 = static_cast<long long>(BH) * N * d / 8;
+    const int blocks = static_cast<int>((n8 + 255) / 256);
+    LaunchTrace trace(kKernBwdConvert, stream);
+    fa::fa_bwd_dq_convert<<<blocks, 256, 0, stream>>>(dq_acc, dq, n8, scale, grad_dtype);
+    if (cudaPeekAtLastError() != cudaSuccess) return FA_ERR_LAUNCH;
+  }
+  return FA_OK;
 }
 
 }  // namespace
@@ -159,8 +298,9 @@ int fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int
   if ((s = device_info(&info)) != FA_OK) return s;
   const int BH = B * H;
   CUtensorMap tq, tk, tv;
-  if (make_tmap(&tq, q, BH, N, d) != FA_OK || make_tmap(&tk, k, BH, N, d) != FA_OK ||
-      make_tmap(&tv, v, BH, N, d) != FA_OK)
+  if (make_tmap_rows(&tq, q, BH, N, d, 128) != FA_OK ||
+      make_tmap_rows(&tk, k, BH, N, d, 128) != FA_OK ||
+      make_tmap_rows(&tv, v, BH, N, d, 128) != FA_OK)
     return FA_ERR_LAUNCH;
   fa::FwdParams p;
   p.o = static_cast<__nv_bfloat16*>(o);
@@ -200,9 +340,8 @@ int fa_bwd(const void* q, const void* k, const void* v, const void* o, const voi
   if (workspace_bytes < fa::bwd_workspace_bytes(B, H, N, d)) return FA_ERR_WORKSPACE;
   DeviceInfo* info = nullptr;
   if ((s = device_info(&info)) != FA_OK) return s;
-  return fa::launch_bwd(q, k, v, o, dO, lse, dq, dk, dv, B, H, N, d, scale, causal != 0,
-                        workspace, grad_dtype, info->sms, info->status,
-                        reinterpret_cast<cudaStream_t>(stream), g_encode);
+  return launch_bwd(q, k, v, o, dO, lse, dq, dk, dv, B, H, N, d, scale, causal != 0, workspace,
+                    grad_dtype, info->sms, info->status, reinterpret_cast<cudaStream_t>(stream));
 }
 
 int fa_check_device_errors(fa_stream_t stream) {
@@ -218,6 +357,43 @@ int fa_check_device_errors(fa_stream_t stream) {
   if (host & fa::kDevTimeout) return FA_ERR_TIMEOUT;
   if (host & fa::kDevAssert) return FA_ERR_DEVICE_ASSERT;
   return FA_OK;
+}
+
+int fa_trace_start(void) {
+  std::lock_guard<std::mutex> lock(g_trace_mu);
+  g_trace.clear();
+  for (int dev = 0; dev < kMaxDevices; ++dev) g_event_used[dev] = 0;
+  g_trace_on = true;
+  return FA_OK;
+}
+
+int fa_trace_stop(int n_kernels, int* launches, double* total_ms) {
+  std::lock_guard<std::mutex> lock(g_trace_mu);
+  g_trace_on = false;
+  if (n_kernels < 0 || (n_kernels > 0 && (!launches || !total_ms))) return FA_ERR_NULL;
+  for (int k = 0; k < n_kernels; ++k) {
+    launches[k] = 0;
+    total_ms[k] = 0.0;
+  }
+  int rc = FA_OK;
+  for (const TraceRec& r : g_trace) {
+    float ms = 0.f;
+    if (cudaEventSynchronize(r.stop) != cudaSuccess ||
+        cudaEventElapsedTime(&ms, r.start, r.stop) != cudaSuccess) {
+      rc = FA_ERR_LAUNCH;
+      continue;
+    }
+    if (r.kernel < n_kernels) {
+      launches[r.kernel] += 1;
+      total_ms[r.kernel] += ms;
+    }
+  }
+  g_trace.clear();
+  return rc;
+}
+
+const char* fa_trace_kernel_name(int kernel) {
+  return (kernel >= 0 && kernel < kNumKernels) ? kKernelNames[kernel] : "unknown";
 }
 
 }  // extern "C"

@@ -18,11 +18,10 @@
 // the A operand of O_i += P_i V straight from TMEM.  One thread owns one row,
 // so row max and row sum need no shuffles.
 //
-// A work unit is (b*H+h, pair of 128-row Q tiles); units are visited longest
-// first when causal, and CTAs stride through them (persistent grid of
-// min(units, SMs) CTAs), so no partial last wave of whole CTAs is left
-// (wave quantization, "CS336 Lecture 5 · GPUs, TPUs" notes, section
-// "波次量化").
+// A work unit is (b*H+h, pair of 128-row Q tiles); units are sorted longest
+// first when causal and dealt to a persistent grid of min(units, SMs) CTAs
+// in a snake order, so no partial last wave of whole CTAs is left (wave
+// quantization, "CS336 Lecture 5 · GPUs, TPUs" notes, section "波次量化").
 //
 // Causal masking is by tile skipping: Q tile i only visits key tiles up to
 // its diagonal, and only the diagonal tile (and a ragged last key tile) pays
@@ -87,6 +86,19 @@ __device__ __forceinline__ FwdUnit fwd_decode(const FwdParams& p, int w) {
   return u;
 }
 
+// Static "snake" assignment of work units to persistent CTAs: in round r,
+// CTA c takes unit r*G + c when r is even and r*G + (G-1-c) when r is odd
+// (G = gridDim.x).  With units sorted longest first this keeps every CTA's
+// total close to the mean.  Returns -1 past the end; `r` is the round.
+__device__ __forceinline__ int snake_unit(int r, int n_units) {
+  const int G = gridDim.x, c = blockIdx.x;
+  const int w = r * G + ((r & 1) ? (G - 1 - c) : c);
+  return w < n_units ? w : -1;
+}
+__device__ __forceinline__ int snake_rounds(int n_units) {
+  return (n_units + gridDim.x - 1) / gridDim.x;
+}
+
 // Wait on an mbarrier from one thread; false (and the CTA's abort flag set)
 // if the wait timed out or another role already aborted.
 __device__ __forceinline__ bool wait1(uint64_t* bar, uint32_t parity, FwdBarriers* b,
@@ -114,7 +126,9 @@ __device__ void fwd_producer(const CUtensorMap* tm_q, const CUtensorMap* tm_k,
                              FwdBarriers* b, int& kc, int& vc, int& units) {
   using L = FwdLayout<D>;
   constexpr int S = L::kStages;
-  for (int w = blockIdx.x; w < p.n_units; w += gridDim.x) {
+  for (int r = 0, nr = snake_rounds(p.n_units); r < nr; ++r) {
+    const int w = snake_unit(r, p.n_units);
+    if (w < 0) continue;
     const FwdUnit u = fwd_decode<CAUSAL>(p, w);
     if (units > 0 && !wait1(&b->q_empty, (units - 1) & 1, b, p.status)) return;
     mbar_arrive_expect_tx(&b->q_full, 2 * L::kTileBytes);
@@ -183,7 +197,9 @@ __device__ void fwd_mma(const FwdParams& p, uint8_t* smem, FwdBarriers* b, uint3
   const uint32_t qs[2] = {sb + L::kQ0, sb + L::kQ1};
   int qc = 0, kc = 0, vc = 0;
   int pc[2] = {0, 0};
-  for (int w = blockIdx.x; w < p.n_units; w += gridDim.x) {
+  for (int r = 0, nr = snake_rounds(p.n_units); r < nr; ++r) {
+    const int w = snake_unit(r, p.n_units);
+    if (w < 0) continue;
     const FwdUnit u = fwd_decode<CAUSAL>(p, w);
     const int nk0 = u.nk0, nk1 = u.nk1, nk = u.nk1;
     if (!wait1(&b->q_full, qc & 1, b, p.status)) return;
@@ -264,7 +280,9 @@ __device__ void fwd_softmax(const FwdParams& p, FwdBarriers* b, uint32_t tmem, i
   const float sl2 = p.scale_log2;
   const int N = p.N;
   int sc = 0, oc = 0;
-  for (int w = blockIdx.x; w < p.n_units; w += gridDim.x) {
+  for (int r = 0, nr = snake_rounds(p.n_units); r < nr; ++r) {
+    const int w = snake_unit(r, p.n_units);
+    if (w < 0) continue;
     const FwdUnit u = fwd_decode<CAUSAL>(p, w);
     const int nk = wg ? u.nk1 : u.nk0;
     const int tile_row0 = u.q0 + wg * 128;

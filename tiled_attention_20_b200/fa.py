@@ -25,7 +25,9 @@ STATUS_NAMES = {
 }
 
 EXPORTED = ["fa_fwd", "fa_bwd", "fa_bwd_workspace_size", "fa_strerror",
-            "fa_check_device_errors", "fa_launch_shape"]
+            "fa_check_device_errors", "fa_launch_shape", "fa_trace_start", "fa_trace_stop",
+            "fa_trace_kernel_name"]
+KERNEL_IDS = {0: "fa_fwd_kernel", 1: "fa_bwd_prep", 2: "fa_bwd_kernel", 3: "fa_bwd_dq_convert"}
 
 
 class FAError(RuntimeError):
@@ -61,6 +63,12 @@ def load(path: str = LIB_PATH):
         lib.fa_launch_shape.argtypes = [_i, _i, _i, _i, _i, _i,
                                         ctypes.POINTER(_i), ctypes.POINTER(_i)]
         lib.fa_launch_shape.restype = _i
+        lib.fa_trace_start.argtypes = []
+        lib.fa_trace_start.restype = _i
+        lib.fa_trace_stop.argtypes = [_i, ctypes.POINTER(_i), ctypes.POINTER(ctypes.c_double)]
+        lib.fa_trace_stop.restype = _i
+        lib.fa_trace_kernel_name.argtypes = [_i]
+        lib.fa_trace_kernel_name.restype = ctypes.c_char_p
         _lib = lib
     return _lib
 
@@ -155,3 +163,18 @@ def launch_shape(pass_: int, B, H, N, d, causal=False):
     _check(load().fa_launch_shape(pass_, B, H, N, d, int(bool(causal)), ctypes.byref(ctas),
                                   ctypes.byref(units)), "fa_launch_shape")
     return ctas.value, units.value
+
+
+def trace_start() -> None:
+    """Start bracketing every library launch with CUDA events."""
+    _check(load().fa_trace_start(), "fa_trace_start")
+
+
+def trace_stop() -> dict:
+    """Stop tracing; {kernel name: (launches, total ms)} for kernels that ran."""
+    n = len(KERNEL_IDS)
+    launches = (_i * n)()
+    ms = (ctypes.c_double * n)()
+    _check(load().fa_trace_stop(n, launches, ms), "fa_trace_stop")
+    return {load().fa_trace_kernel_name(k).decode(): (launches[k], ms[k])
+            for k in range(n) if launches[k]}
