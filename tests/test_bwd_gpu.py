@@ -85,15 +85,21 @@ def test_long_context_distribution_small():
 @pytest.mark.parametrize("causal", [False, True])
 def test_gradient_sum_rules_on_gpu(causal):
     """Key-shift invariance gives sum_j dK_j = 0; rows of P summing to one give
-    sum_j dV_j = sum_i dO_i.  Checked on fp32 gradient outputs for every head."""
-    (q, k, v, dO), _, (dq, dk, dv) = _run(2, 4, 700, 128, causal, seed=3,
-                                          grad_dtype=torch.float32)
-    sdk = np64(dk).sum(axis=2)
-    sdv = np64(dv).sum(axis=2)
-    sdo = np64(dO).sum(axis=2)
-    scale_dk = np.abs(np64(dk)).sum(axis=2).max()
-    assert np.abs(sdk).max() <= 1e-2 * max(1.0, scale_dk / 100), np.abs(sdk).max()
-    np.testing.assert_allclose(sdv, sdo, rtol=0, atol=0.1)
+    sum_j dV_j = sum_i dO_i.  Checked per head and column on fp32 gradient
+    outputs, with bounds from the rounding model of the kernel: the bf16
+    operands P and dS carry a relative error of at most 2^-9 each, and D is
+    formed from the bf16 output O, so sum_j dS_ij is off by at most
+    2^-9 sum_c |dO_ic O_ic|.  The bounds below are those, doubled."""
+    (q, k, v, dO), (o, _), (dq, dk, dv) = _run(2, 4, 700, 128, causal, seed=3,
+                                               grad_dtype=torch.float32)
+    scale = 1 / np.sqrt(128)
+    dk64, dv64, dO64, q64, o64 = np64(dk), np64(dv), np64(dO), np64(q), np64(o)
+    u = 2.0 ** -9
+    dd = np.abs(dO64 * o64).sum(axis=3, keepdims=True)          # [B,H,N,1]
+    bound_k = 2 * (u * np.abs(dk64).sum(axis=2) + scale * u * (dd * np.abs(q64)).sum(axis=2))
+    assert (np.abs(dk64.sum(axis=2)) <= bound_k).all(), np.abs(dk64.sum(axis=2)).max()
+    bound_v = 2 * u * np.abs(dO64).sum(axis=2) + 1e-6
+    assert (np.abs(dv64.sum(axis=2) - dO64.sum(axis=2)) <= bound_v).all()
 
 
 def test_workspace_contents_do_not_matter():

@@ -413,8 +413,7 @@ __device__ void bwd_compute(const BwdParams& p, uint8_t* smem, BwdBarriers* b, u
 #pragma unroll
       for (int h = 0; h < 2; ++h) {
         uint32_t rs[32], rp[32];
-        tmem_ld_x32(tS + 32 * h, rs);
-        tmem_ld_x32(tdP + 32 * h, rp);
+        tmem_ld_x32_pair(tS + 32 * h, tdP + 32 * h, rs, rp);
         float pr[32];
 #pragma unroll
         for (int c4 = 0; c4 < 8; ++c4) {

@@ -2,6 +2,7 @@
 // validation, TMA descriptor construction, persistent-grid sizing and kernel
 // launches.  Every step of the computation runs in the kernels; this file
 // only prepares launches.
+#include <cfloat>
 #include <cmath>
 #include <cstdint>
 #include <cstring>
@@ -144,6 +145,12 @@ int launch_fwd(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& 
                const fa::FwdParams& p, int ctas, cudaStream_t stream) {
   auto kern = fa::fa_fwd_kernel<D, CAUSAL>;
   const int smem = fa::FwdLayout<D>::kSmemBytes;
+  // The kernel moves registers between warpgroups; its split assumes the
+  // launch allocation it was compiled for.  Refuse to launch otherwise
+  // (a larger request than the block holds would never be granted).
+  cudaFuncAttributes attr;
+  if (cudaFuncGetAttributes(&attr, kern) != cudaSuccess || attr.numRegs != fa::kFwdLaunchRegs)
+    return FA_ERR_LAUNCH;
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
     return FA_ERR_LAUNCH;
   LaunchTrace trace(kKernFwd, stream);
@@ -309,7 +316,10 @@ int fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int
   p.N = N;
   p.n_qt2 = (N + 255) / 256;
   p.n_units = fwd_units(B, H, N);
-  p.scale_log2 = scale * 1.4426950408889634f;
+  // Masked scores are -inf before scaling; a zero scale would turn them into
+  // NaN.  FLT_MIN keeps them at -inf while every finite score still scales
+  // to zero, so scale = 0 gives exactly uniform weights.
+  p.scale_log2 = std::fmax(scale * 1.4426950408889634f, FLT_MIN);
   p.status = info->status;
   const int ctas = p.n_units < info->sms ? p.n_units : info->sms;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);

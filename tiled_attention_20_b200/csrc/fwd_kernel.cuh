@@ -60,6 +60,16 @@ struct FwdLayout {
   static constexpr int kSmemBytes = kBar + kBarBytes + 1024;  // + manual 1024-B alignment
 };
 
+// Registers per thread: the kernel is launched with kFwdLaunchRegs; then
+// warpgroup 0 (producer, MMA issuer, two idle warps) gives registers up to
+// the two softmax warpgroups, which hold a 128-score row per thread.
+// 128 * kFwdCtlRegs + 256 * kFwdSoftmaxRegs == 384 * kFwdLaunchRegs.
+constexpr int kFwdLaunchRegs = 168;
+constexpr int kFwdCtlRegs = 72;
+constexpr int kFwdSoftmaxRegs = 216;
+static_assert(128 * kFwdCtlRegs + 256 * kFwdSoftmaxRegs <= 384 * kFwdLaunchRegs,
+              "register split exceeds the launch allocation");
+
 struct FwdBarriers {
   uint64_t q_full, q_empty;
   uint64_t k_full[4], k_empty[4], v_full[4], v_empty[4];
@@ -303,13 +313,15 @@ __device__ void fwd_softmax(const FwdParams& p, FwdBarriers* b, uint32_t tmem, i
 #pragma unroll
         for (int c = 0; c < 128; ++c) s[c] = (key0 + c < lim) ? s[c] : -INFINITY;
       }
-      float mx[8];
+      // Row maximum: four independent chains of three-input max.
+      float mx[4];
 #pragma unroll
-      for (int i = 0; i < 8; ++i) mx[i] = s[i];
+      for (int k4 = 0; k4 < 4; ++k4) {
+        mx[k4] = fmaxf(s[32 * k4], s[32 * k4 + 1]);
 #pragma unroll
-      for (int c = 8; c < 128; ++c) mx[c & 7] = fmaxf(mx[c & 7], s[c]);
-      float m_tile = fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])),
-                           fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7])));
+        for (int c = 32 * k4 + 2; c < 32 * k4 + 32; c += 2) mx[k4] = max3(mx[k4], s[c], s[c + 1]);
+      }
+      float m_tile = max3(mx[0], mx[1], fmaxf(mx[2], mx[3]));
       m_tile *= sl2;
       const bool need = m_tile > m_used + 8.0f;
       if (__any_sync(0xffffffffu, need)) {
@@ -318,29 +330,58 @@ __device__ void fwd_softmax(const FwdParams& p, FwdBarriers* b, uint32_t tmem, i
         l *= alpha;
         if (j > 0) {
 #pragma unroll
-          for (int c0 = 0; c0 < D; c0 += 32) {
-            uint32_t o[32];
-            tmem_ld_x32(tO + c0, o);
+          for (int c0 = 0; c0 < D; c0 += 16) {
+            uint32_t o[16];
+            tmem_ld_x16(tO + c0, o);
 #pragma unroll
-            for (int c = 0; c < 32; ++c) o[c] = __float_as_uint(__uint_as_float(o[c]) * alpha);
-            tmem_st_x32(tO + c0, o);
+            for (int c = 0; c < 16; ++c) o[c] = __float_as_uint(__uint_as_float(o[c]) * alpha);
+            tmem_st_x16(tO + c0, o);
           }
         }
         m_used = m_new;
       }
       const float mb = (m_used == -INFINITY) ? 0.f : m_used;
-      float rs[4] = {0.f, 0.f, 0.f, 0.f};
-      uint32_t pk[64];
+      const float2 sl2v = make_float2(sl2, sl2);
+      const float2 nmb = make_float2(-mb, -mb);
+      float2 rs[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f),
+                      make_float2(0.f, 0.f)};
+      // P in two halves of 64 keys; each half is stored as soon as it is
+      // packed (S is already in registers, so overwriting it is safe).  On
+      // unmasked tiles 3 of every 8 pairs take the polynomial exp2 on the
+      // FMA pipe and the rest the MUFU unit; masked tiles (which hold -inf)
+      // use the MUFU unit throughout so masked probabilities are exactly 0.
+      if (need_mask) {
 #pragma unroll
-      for (int c = 0; c < 128; c += 2) {
-        const float p0 = ex2_approx(fmaf(s[c], sl2, -mb));
-        const float p1 = ex2_approx(fmaf(s[c + 1], sl2, -mb));
-        rs[(c >> 1) & 3] += p0 + p1;
-        pk[c >> 1] = pack_bf16x2(p0, p1);
+        for (int h = 0; h < 2; ++h) {
+          uint32_t pk[32];
+#pragma unroll
+          for (int q2 = 0; q2 < 32; ++q2) {
+            const int c = 64 * h + 2 * q2;
+            const float2 x = fma2(make_float2(s[c], s[c + 1]), sl2v, nmb);
+            const float2 pp = make_float2(ex2_approx(x.x), ex2_approx(x.y));
+            rs[q2 & 3] = add2(rs[q2 & 3], pp);
+            pk[q2] = pack_bf16x2(pp.x, pp.y);
+          }
+          tmem_st_x32(tS + 32 * h, pk);
+        }
+      } else {
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          uint32_t pk[32];
+#pragma unroll
+          for (int q2 = 0; q2 < 32; ++q2) {
+            const int c = 64 * h + 2 * q2;
+            const float2 x = fma2(make_float2(s[c], s[c + 1]), sl2v, nmb);
+            const float2 pp = ((q2 & 7) < 3) ? exp2_poly2(x)
+                                             : make_float2(ex2_approx(x.x), ex2_approx(x.y));
+            rs[q2 & 3] = add2(rs[q2 & 3], pp);
+            pk[q2] = pack_bf16x2(pp.x, pp.y);
+          }
+          tmem_st_x32(tS + 32 * h, pk);
+        }
       }
-      l += (rs[0] + rs[1]) + (rs[2] + rs[3]);
-      tmem_st_x32(tS, pk);
-      tmem_st_x32(tS + 32, pk + 32);
+      const float2 rsum = add2(add2(rs[0], rs[1]), add2(rs[2], rs[3]));
+      l += rsum.x + rsum.y;
       tmem_st_wait();
       tc_fence_before();
       mbar_arrive(&b->p_full[wg]);
@@ -414,35 +455,38 @@ __global__ void __launch_bounds__(384, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = b->tmem_base;
-
-  if (warp == 0) {
-    if (lane_id() == 0) {
-      int kc = 0, vc = 0, units = 0;
-      fwd_producer<D, CAUSAL>(&tm_q, &tm_k, &tm_v, p, smem, b, kc, vc, units);
-      // Wait for every TMA load this thread armed (all long complete on the
-      // normal path) so no copy is in flight when the CTA exits.
-      constexpr int S = L::kStages;
-      if (units > 0) mbar_wait(&b->q_full, (units - 1) & 1, p.status);
-      for (int st = 0; st < S; ++st) {
-        const int nk = kc / S + (st < kc % S ? 1 : 0);
-        const int nv = vc / S + (st < vc % S ? 1 : 0);
-        if (nk > 0) mbar_wait(&b->k_full[st], (nk - 1) & 1, p.status);
-        if (nv > 0) mbar_wait(&b->v_full[st], (nv - 1) & 1, p.status);
-      }
-    }
-    __syncwarp();
-  } else if (warp == 1) {
-    if (lane_id() == 0) {
-      fwd_mma<D, CAUSAL>(p, smem, b, tmem);
-      // Drain every MMA this thread issued before TMEM is released.
-      mma_commit(&b->mma_done);
-      mbar_wait(&b->mma_done, 0, p.status);
-    }
-    __syncwarp();
-  } else if (warp >= 4) {
+  if (warp >= 4) {
+    // Softmax warpgroups: take the registers warpgroup 0 gives up.
+    regs_increase<kFwdSoftmaxRegs>();
     fwd_softmax<D, CAUSAL>(p, b, tmem, (warp - 4) >> 2);
+  } else {
+    regs_decrease<kFwdCtlRegs>();
+    if (warp == 0) {
+      if (lane_id() == 0) {
+        int kc = 0, vc = 0, units = 0;
+        fwd_producer<D, CAUSAL>(&tm_q, &tm_k, &tm_v, p, smem, b, kc, vc, units);
+        // Wait for every TMA load this thread armed (all long complete on the
+        // normal path) so no copy is in flight when the CTA exits.
+        constexpr int S = L::kStages;
+        if (units > 0) mbar_wait(&b->q_full, (units - 1) & 1, p.status);
+        for (int st = 0; st < S; ++st) {
+          const int nk = kc / S + (st < kc % S ? 1 : 0);
+          const int nv = vc / S + (st < vc % S ? 1 : 0);
+          if (nk > 0) mbar_wait(&b->k_full[st], (nk - 1) & 1, p.status);
+          if (nv > 0) mbar_wait(&b->v_full[st], (nv - 1) & 1, p.status);
+        }
+      }
+      __syncwarp();
+    } else if (warp == 1) {
+      if (lane_id() == 0) {
+        fwd_mma<D, CAUSAL>(p, smem, b, tmem);
+        // Drain every MMA this thread issued before TMEM is released.
+        mma_commit(&b->mma_done);
+        mbar_wait(&b->mma_done, 0, p.status);
+      }
+      __syncwarp();
+    }
   }
-
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
