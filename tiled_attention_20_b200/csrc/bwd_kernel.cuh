@@ -33,8 +33,8 @@
 //               dQ^T = K^T dS^T).  At the end of a unit warpgroup 0 writes
 //               dV and warpgroup 1 writes dK.
 //   warps 12-15 dQ drain: one thread per head-dimension column; moves dQ^T
-//               from TMEM to shared memory and adds it into the fp32
-//               accumulator in global memory with bulk reduce-add copies.
+//               from TMEM through shared memory into the fp32 accumulator in
+//               global memory with bulk reduce-add copies.
 // Work units are ordered in groups of a few heads (so the dQ accumulator,
 // Q and dO of the heads in flight stay in L2), longest first (ascending K/V
 // block) within a group, and handed out dynamically.
@@ -95,8 +95,8 @@ struct BwdLayout {
   static constexpr int kQ = 2 * kKVBytes;
   static constexpr int kDO = kQ + kQStages * kQBytes;
   static constexpr int kDs = kDO + kQStages * kQBytes;
-  static constexpr int kStage = kDs + 2 * kDsBytes;
-  static constexpr int kLse = kStage + kStageBytes;  // [3][64] fp32
+  static constexpr int kStage = kDs + 2 * kDsBytes;  // two dQ staging buffers
+  static constexpr int kLse = kStage + 2 * kStageBytes;  // [3][64] fp32
   static constexpr int kDv = kLse + kQStages * 256;   // [3][64] fp32
   static constexpr int kBar = kDv + kQStages * 256;
   static constexpr int kBarBytes = 512;
@@ -107,6 +107,17 @@ struct BwdLayout {
   static constexpr uint32_t kTS = 2 * D;         // + 64 s
   static constexpr uint32_t kTdP = 2 * D + 128;  // + 64 s
 };
+
+// Registers per thread: launched with kBwdLaunchRegs (512 threads), then
+// warpgroup 0 (producer, MMA issuer, two idle warps) and the drain
+// warpgroup give registers to the two compute warpgroups.
+constexpr int kBwdLaunchRegs = 128;
+constexpr int kBwdCtlRegs = 64;
+constexpr int kBwdComputeRegs = 176;
+constexpr int kBwdDrainRegs = 80;
+static_assert(128 * kBwdCtlRegs + 256 * kBwdComputeRegs + 128 * kBwdDrainRegs <=
+                  512 * kBwdLaunchRegs,
+              "register split exceeds the launch allocation");
 
 constexpr int kUnitRing = 4;
 // Consumers of the unit ring, counted in arrivals: the MMA thread, the 8
@@ -206,6 +217,9 @@ __device__ __forceinline__ void bulk_commit() {
 }
 __device__ __forceinline__ void bulk_wait_read0() {
   asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
+}
+__device__ __forceinline__ void bulk_wait_read1() {
+  asm volatile("cp.async.bulk.wait_group.read 1;" ::: "memory");
 }
 __device__ __forceinline__ void bulk_wait0() {
   asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
@@ -410,44 +424,56 @@ __device__ void bwd_compute(const BwdParams& p, uint8_t* smem, BwdBarriers* b, u
       const float4* lse4 = reinterpret_cast<const float4*>(smem + L::kLse + qs * 256);
       const float4* dv4 = reinterpret_cast<const float4*>(smem + L::kDv + qs * 256);
       const bool diag = CAUSAL && q0 < u.j * 128 + 127;
+      uint32_t rs[64], rp[64];
+      tmem_ld_x64_pair(tS, tdP, rs, rp);
+      const float2 sl2v = make_float2(sl2, sl2);
+      // P^T = exp2(scale*log2e * S^T - lse*log2e), stored to TMEM as bf16
+      // pairs; rs[] keeps P in fp32 for dS.
+      {
+        uint32_t pk[32];
 #pragma unroll
-      for (int h = 0; h < 2; ++h) {
-        uint32_t rs[32], rp[32];
-        tmem_ld_x32_pair(tS + 32 * h, tdP + 32 * h, rs, rp);
-        float pr[32];
-#pragma unroll
-        for (int c4 = 0; c4 < 8; ++c4) {
-          const float4 l4 = lse4[8 * h + c4];
-          pr[4 * c4 + 0] = ex2_approx(fmaf(__uint_as_float(rs[4 * c4 + 0]), sl2, -l4.x));
-          pr[4 * c4 + 1] = ex2_approx(fmaf(__uint_as_float(rs[4 * c4 + 1]), sl2, -l4.y));
-          pr[4 * c4 + 2] = ex2_approx(fmaf(__uint_as_float(rs[4 * c4 + 2]), sl2, -l4.z));
-          pr[4 * c4 + 3] = ex2_approx(fmaf(__uint_as_float(rs[4 * c4 + 3]), sl2, -l4.w));
-        }
-        if (diag) {
-#pragma unroll
-          for (int c = 0; c < 32; ++c) pr[c] = (key <= q0 + 32 * h + c) ? pr[c] : 0.f;
-        }
-        uint32_t pk[16];
-#pragma unroll
-        for (int c = 0; c < 16; ++c) pk[c] = pack_bf16x2(pr[2 * c], pr[2 * c + 1]);
-        tmem_st_x16(tS + 16 * h, pk);
-#pragma unroll
-        for (int piece = 0; piece < 4; ++piece) {  // 8 queries = 16 bytes per piece
-          const float4 da = dv4[8 * h + 2 * piece], db = dv4[8 * h + 2 * piece + 1];
-          const float d8[8] = {da.x, da.y, da.z, da.w, db.x, db.y, db.z, db.w};
-          uint32_t w4[4];
-#pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            const int c = piece * 8 + 2 * e;
-            const float ds0 = pr[c] * (__uint_as_float(rp[c]) - d8[2 * e]);
-            const float ds1 = pr[c + 1] * (__uint_as_float(rp[c + 1]) - d8[2 * e + 1]);
-            w4[e] = pack_bf16x2(ds0, ds1);
+        for (int c4 = 0; c4 < 16; ++c4) {
+          const float4 l4 = lse4[c4];
+          const int c = 4 * c4;
+          const float2 x0 = fma2(make_float2(__uint_as_float(rs[c]), __uint_as_float(rs[c + 1])),
+                                 sl2v, make_float2(-l4.x, -l4.y));
+          const float2 x1 = fma2(make_float2(__uint_as_float(rs[c + 2]), __uint_as_float(rs[c + 3])),
+                                 sl2v, make_float2(-l4.z, -l4.w));
+          float p0 = ex2_approx(x0.x), p1 = ex2_approx(x0.y), p2 = ex2_approx(x1.x),
+                p3 = ex2_approx(x1.y);
+          if (diag) {
+            p0 = (key <= q0 + c) ? p0 : 0.f;
+            p1 = (key <= q0 + c + 1) ? p1 : 0.f;
+            p2 = (key <= q0 + c + 2) ? p2 : 0.f;
+            p3 = (key <= q0 + c + 3) ? p3 : 0.f;
           }
-          // 128-byte swizzle: 16-byte piece index XOR (row mod 8).
-          const int pc = 4 * h + piece;
-          *reinterpret_cast<uint4*>(ds_row + ((pc ^ (t & 7)) << 4)) =
-              make_uint4(w4[0], w4[1], w4[2], w4[3]);
+          rs[c] = __float_as_uint(p0);
+          rs[c + 1] = __float_as_uint(p1);
+          rs[c + 2] = __float_as_uint(p2);
+          rs[c + 3] = __float_as_uint(p3);
+          pk[2 * c4] = pack_bf16x2(p0, p1);
+          pk[2 * c4 + 1] = pack_bf16x2(p2, p3);
         }
+        tmem_st_x32(tS, pk);
+      }
+      // dS^T = P^T (dP^T - D), to shared memory as bf16 in the 128-byte
+      // swizzled layout the tensor core reads.
+#pragma unroll
+      for (int piece = 0; piece < 8; ++piece) {  // 8 queries = 16 bytes per piece
+        const float4 da = dv4[2 * piece], db = dv4[2 * piece + 1];
+        const int c = 8 * piece;
+        uint32_t w4[4];
+        const float2 d2[4] = {make_float2(da.x, da.y), make_float2(da.z, da.w),
+                              make_float2(db.x, db.y), make_float2(db.z, db.w)};
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const float2 pp = make_float2(__uint_as_float(rs[c + 2 * e]), __uint_as_float(rs[c + 2 * e + 1]));
+          const float2 dp = make_float2(__uint_as_float(rp[c + 2 * e]), __uint_as_float(rp[c + 2 * e + 1]));
+          const float2 ds = mul2(pp, add2(dp, make_float2(-d2[e].x, -d2[e].y)));
+          w4[e] = pack_bf16x2(ds.x, ds.y);
+        }
+        *reinterpret_cast<uint4*>(ds_row + ((piece ^ (t & 7)) << 4)) =
+            make_uint4(w4[0], w4[1], w4[2], w4[3]);
       }
       tmem_st_wait();
       tc_fence_before();
@@ -495,6 +521,10 @@ __device__ void bwd_compute(const BwdParams& p, uint8_t* smem, BwdBarriers* b, u
 }
 
 // ---------------------------------------------------------------- dQ drain
+// Moves dQ^T of each Q block from TMEM to registers, stages it row-major in
+// shared memory (32 rows at a time, two buffers) and adds it into the fp32
+// accumulator with bulk reduce-add copies, one in flight while the other
+// buffer fills.
 template <int D, bool CAUSAL>
 __device__ void bwd_drain(const BwdParams& p, uint8_t* smem, BwdBarriers* b, uint32_t tmem) {
   using L = BwdLayout<D>;
@@ -506,7 +536,6 @@ __device__ void bwd_drain(const BwdParams& p, uint8_t* smem, BwdBarriers* b, uin
   const bool valid = (D == 128) || (ln < 16);
   const int dcol = (D == 128) ? t : (quarter * 16 + ln);
   const bool issuer = (t == 0);
-  float* stage = reinterpret_cast<float*>(smem + L::kStage);
   int g = 0, rc = 0;
   for (;;) {
     const int w = next_unit_warp(b, rc, p.status);
@@ -526,7 +555,8 @@ __device__ void bwd_drain(const BwdParams& p, uint8_t* smem, BwdBarriers* b, uin
       mbar_arrive(&b->dq_empty[s]);
 #pragma unroll
       for (int half = 0; half < 2; ++half) {
-        if (issuer) bulk_wait_read0();  // the previous reduce has read the stage
+        float* stage = reinterpret_cast<float*>(smem + L::kStage + half * L::kStageBytes);
+        if (issuer) bulk_wait_read1();  // this buffer's previous reduce has read it
         named_bar_sync(1, 128);
         if (valid) {
 #pragma unroll
@@ -538,11 +568,10 @@ __device__ void bwd_drain(const BwdParams& p, uint8_t* smem, BwdBarriers* b, uin
         if (issuer) {
           const int r0 = q0 + half * L::kStageRows;
           const int rows = min(L::kStageRows, p.N - r0);
-          if (rows > 0) {
+          if (rows > 0)
             bulk_reduce_add_f32(p.dq_acc + (static_cast<size_t>(u.bh) * p.N + r0) * D, stage,
                                 rows * D * 4);
-            bulk_commit();
-          }
+          bulk_commit();  // an empty group keeps the two-buffer accounting exact
         }
       }
     }
@@ -602,30 +631,35 @@ __global__ void __launch_bounds__(512, 1)
   tc_fence_after();
   const uint32_t tmem = b->tmem_base;
 
-  if (warp == 0) {
-    if (lane_id() == 0) {
-      int qc = 0, kvc = 0;
-      bwd_producer<D, CAUSAL>(&tm_q, &tm_k, &tm_v, &tm_do, p, smem, b, qc, kvc);
-      // No copy may be in flight when the CTA exits.
-      constexpr int QS = L::kQStages;
-      if (kvc > 0) mbar_wait(&b->kv_full, (kvc - 1) & 1, p.status);
-      for (int st = 0; st < QS; ++st) {
-        const int n = qc / QS + (st < qc % QS ? 1 : 0);
-        if (n > 0) mbar_wait(&b->q_full[st], (n - 1) & 1, p.status);
-      }
-    }
-    __syncwarp();
-  } else if (warp == 1) {
-    if (lane_id() == 0) {
-      bwd_mma<D, CAUSAL>(p, smem, b, tmem);
-      mma_commit(&b->mma_done);
-      mbar_wait(&b->mma_done, 0, p.status);
-    }
-    __syncwarp();
-  } else if (warp >= 4 && warp < 12) {
+  if (warp >= 4 && warp < 12) {
+    regs_increase<kBwdComputeRegs>();
     bwd_compute<D, CAUSAL>(p, smem, b, tmem, (warp - 4) >> 2);
   } else if (warp >= 12) {
+    regs_decrease<kBwdDrainRegs>();
     bwd_drain<D, CAUSAL>(p, smem, b, tmem);
+  } else {
+    regs_decrease<kBwdCtlRegs>();
+    if (warp == 0) {
+      if (lane_id() == 0) {
+        int qc = 0, kvc = 0;
+        bwd_producer<D, CAUSAL>(&tm_q, &tm_k, &tm_v, &tm_do, p, smem, b, qc, kvc);
+        // No copy may be in flight when the CTA exits.
+        constexpr int QS = L::kQStages;
+        if (kvc > 0) mbar_wait(&b->kv_full, (kvc - 1) & 1, p.status);
+        for (int st = 0; st < QS; ++st) {
+          const int n = qc / QS + (st < qc % QS ? 1 : 0);
+          if (n > 0) mbar_wait(&b->q_full[st], (n - 1) & 1, p.status);
+        }
+      }
+      __syncwarp();
+    } else if (warp == 1) {
+      if (lane_id() == 0) {
+        bwd_mma<D, CAUSAL>(p, smem, b, tmem);
+        mma_commit(&b->mma_done);
+        mbar_wait(&b->mma_done, 0, p.status);
+      }
+      __syncwarp();
+    }
   }
   tc_fence_before();
   __syncthreads();

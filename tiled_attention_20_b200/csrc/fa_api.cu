@@ -181,6 +181,10 @@ int launch_bwd_main(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensor
                     cudaStream_t stream) {
   auto kern = fa::fa_bwd_kernel<D, CAUSAL>;
   const int smem = fa::BwdLayout<D>::kSmemBytes;
+  // The register split between warpgroups assumes this launch allocation.
+  cudaFuncAttributes attr;
+  if (cudaFuncGetAttributes(&attr, kern) != cudaSuccess || attr.numRegs != fa::kBwdLaunchRegs)
+    return FA_ERR_LAUNCH;
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
     return FA_ERR_LAUNCH;
   LaunchTrace trace(kKernBwd, stream);
