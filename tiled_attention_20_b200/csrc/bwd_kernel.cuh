@@ -489,32 +489,32 @@ __device__ void bwd_compute(const BwdParams& p, uint8_t* smem, BwdBarriers* b, u
     const uint32_t col = s ? L::kTdK : L::kTdV;
     const float mul = s ? p.scale : 1.f;
     void* out = s ? p.dk : p.dv;
+    uint32_t r[D];
+    if (D == 128)
+      tmem_ld_x128(tmem + lane_base + col, r);
+    else
+      tmem_ld_x64(tmem + lane_base + col, r);
+    tc_fence_before();
+    mbar_arrive(&b->acc_empty);  // TMEM read: the next unit may overwrite dK, dV
+    if (valid) {
+      if (p.grad_f32) {
+        float4* dst = reinterpret_cast<float4*>(static_cast<float*>(out) + row * D);
 #pragma unroll
-    for (int c0 = 0; c0 < D; c0 += 32) {
-      uint32_t r[32];
-      tmem_ld_x32(tmem + lane_base + col + c0, r);
-      if (valid) {
-        if (p.grad_f32) {
-          float4* dst = reinterpret_cast<float4*>(static_cast<float*>(out) + row * D + c0);
+        for (int v = 0; v < D / 4; ++v)
+          dst[v] = make_float4(__uint_as_float(r[4 * v]) * mul, __uint_as_float(r[4 * v + 1]) * mul,
+                               __uint_as_float(r[4 * v + 2]) * mul,
+                               __uint_as_float(r[4 * v + 3]) * mul);
+      } else {
+        uint4* dst = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(out) + row * D);
 #pragma unroll
-          for (int v = 0; v < 8; ++v)
-            dst[v] = make_float4(__uint_as_float(r[4 * v]) * mul, __uint_as_float(r[4 * v + 1]) * mul,
-                                 __uint_as_float(r[4 * v + 2]) * mul,
-                                 __uint_as_float(r[4 * v + 3]) * mul);
-        } else {
-          uint4* dst = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(out) + row * D + c0);
-#pragma unroll
-          for (int v = 0; v < 4; ++v)
-            dst[v] = make_uint4(
-                pack_bf16x2(__uint_as_float(r[8 * v + 0]) * mul, __uint_as_float(r[8 * v + 1]) * mul),
-                pack_bf16x2(__uint_as_float(r[8 * v + 2]) * mul, __uint_as_float(r[8 * v + 3]) * mul),
-                pack_bf16x2(__uint_as_float(r[8 * v + 4]) * mul, __uint_as_float(r[8 * v + 5]) * mul),
-                pack_bf16x2(__uint_as_float(r[8 * v + 6]) * mul, __uint_as_float(r[8 * v + 7]) * mul));
-        }
+        for (int v = 0; v < D / 8; ++v)
+          dst[v] = make_uint4(
+              pack_bf16x2(__uint_as_float(r[8 * v + 0]) * mul, __uint_as_float(r[8 * v + 1]) * mul),
+              pack_bf16x2(__uint_as_float(r[8 * v + 2]) * mul, __uint_as_float(r[8 * v + 3]) * mul),
+              pack_bf16x2(__uint_as_float(r[8 * v + 4]) * mul, __uint_as_float(r[8 * v + 5]) * mul),
+              pack_bf16x2(__uint_as_float(r[8 * v + 6]) * mul, __uint_as_float(r[8 * v + 7]) * mul));
       }
     }
-    tc_fence_before();
-    mbar_arrive(&b->acc_empty);
     g += u.n;
     qbase += u.n;
   }
