@@ -58,7 +58,8 @@ typedef enum {
   FA_ERR_TIMEOUT = -7,        /* a device-side wait gave up (reported later) */
   FA_ERR_DEVICE_ASSERT = -8,  /* a device-side consistency check failed */
   FA_ERR_ARCH = -9,           /* the current device is not sm_100 */
-  FA_ERR_ARG = -10            /* scale negative or not finite; bad grad_dtype */
+  FA_ERR_ARG = -10,           /* scale negative or not finite; bad grad_dtype */
+  FA_ERR_NOALLOC_LIMIT = -11  /* fa_bwd_noalloc: scratch need above its fixed maximum */
 } fa_status;
 
 /*
@@ -135,6 +136,37 @@ int fa_launch_shape(int pass, int B, int H, int N, int d, int causal,
 int fa_trace_start(void);
 int fa_trace_stop(int n_kernels, int *launches, double *total_ms);
 const char *fa_trace_kernel_name(int kernel);
+
+/*
+ * Backward for callers that cannot allocate device memory.  (No counterpart
+ * on the pages: this is a packaging variant of fa_bwd.)  Some callers cannot
+ * call cudaMalloc: a plugin inside a host framework that owns every byte of
+ * device memory and gives its plugins none, or a latency-critical path where
+ * cudaMalloc's implicit device synchronisation is not allowed.  This entry
+ * point runs exactly the fa_bwd computation, with the same arguments minus
+ * the workspace, but takes its scratch from a fixed array inside the
+ * library's device image instead of from the caller.
+ *   - Maximum: fa_bwd_workspace_size(B,H,N,d) must not exceed
+ *     FA_BWD_NOALLOC_MAX_SCRATCH (32 MiB, e.g. B*H = 64 heads of N = 1024 at
+ *     d = 64); larger problems return FA_ERR_NOALLOC_LIMIT before anything is
+ *     enqueued.
+ *   - The array exists on every GPU that loads the library and is held until
+ *     the process exits.
+ *   - The first call on a device looks up the array's device address
+ *     (cudaGetSymbolAddress, with that device current); make that first call
+ *     before any stream capture.  The function allocates and frees nothing.
+ *   - All calls on a device share the one array: calls that overlap on the
+ *     GPU (different streams, no ordering between them) race and corrupt each
+ *     other's results.  Order them on one stream or with events.
+ *   - The array keeps the previous call's contents; every part that must
+ *     start at zero is cleared by the call itself.
+ * Returns FA_OK once the kernels are enqueued, or an fa_status error.
+ */
+#define FA_BWD_NOALLOC_MAX_SCRATCH ((size_t)32 << 20)
+int fa_bwd_noalloc(const void *q, const void *k, const void *v, const void *o,
+                   const void *dO, const float *lse, void *dq, void *dk, void *dv,
+                   int B, int H, int N, int d, float scale, int causal,
+                   int grad_dtype, fa_stream_t stream);
 
 #ifdef __cplusplus
 }

@@ -264,6 +264,33 @@ int launch_bwd(const void* q, const void* k, const void* v, const void* o, const
 
 }  // namespace
 
+// ---------------------------------------------------------------- backward without allocation
+// Scratch for fa_bwd_noalloc: a fixed array in the library's device image,
+// present on every GPU that loads the library until the process exits.
+// Host code must not hand this symbol to a kernel: on the host it names a
+// stand-in, not device memory.  Its device address is looked up per device.
+static __device__ __align__(256) unsigned char g_bwd_noalloc_scratch[FA_BWD_NOALLOC_MAX_SCRATCH];
+
+namespace {
+void* g_noalloc_addr[kMaxDevices];  // device address of the scratch, per device
+
+// The scratch's device address on the current device, looked up on the first
+// call there (with that device current) and remembered.
+int noalloc_scratch(void** out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return FA_ERR_LAUNCH;
+  std::lock_guard<std::mutex> lock(g_mu);
+  if (!g_noalloc_addr[dev]) {
+    void* ptr = nullptr;
+    if (cudaGetSymbolAddress(&ptr, g_bwd_noalloc_scratch) != cudaSuccess || ptr == nullptr)
+      return FA_ERR_LAUNCH;
+    g_noalloc_addr[dev] = ptr;
+  }
+  *out = g_noalloc_addr[dev];
+  return FA_OK;
+}
+}  // namespace
+
 extern "C" {
 
 const char* fa_strerror(int status) {
@@ -279,6 +306,8 @@ const char* fa_strerror(int status) {
     case FA_ERR_DEVICE_ASSERT: return "a device-side consistency check failed";
     case FA_ERR_ARCH: return "the current device is not an sm_100 (B200-class) GPU";
     case FA_ERR_ARG: return "invalid argument (scale must be finite and >= 0; grad_dtype 0 or 1)";
+    case FA_ERR_NOALLOC_LIMIT:
+      return "problem needs more backward scratch than fa_bwd_noalloc's fixed maximum";
     default: return "unknown status";
   }
 }
@@ -408,6 +437,29 @@ int fa_trace_stop(int n_kernels, int* launches, double* total_ms) {
 
 const char* fa_trace_kernel_name(int kernel) {
   return (kernel >= 0 && kernel < kNumKernels) ? kKernelNames[kernel] : "unknown";
+}
+
+int fa_bwd_noalloc(const void* q, const void* k, const void* v, const void* o, const void* dO,
+                   const float* lse, void* dq, void* dk, void* dv, int B, int H, int N, int d,
+                   float scale, int causal, int grad_dtype, fa_stream_t stream) {
+  if (!q || !k || !v || !o || !dO || !lse || !dq || !dk || !dv) return FA_ERR_NULL;
+  int s = check_shape(B, H, N, d);
+  if (s != FA_OK) return s;
+  if ((s = check_scale(scale)) != FA_OK) return s;
+  if (grad_dtype != 0 && grad_dtype != 1) return FA_ERR_ARG;
+  const void* ptrs[] = {q, k, v, o, dO, lse, dq, dk, dv};
+  for (const void* ptr : ptrs)
+    if (!aligned16(ptr)) return FA_ERR_ALIGN;
+  if (fa::bwd_workspace_bytes(B, H, N, d) > FA_BWD_NOALLOC_MAX_SCRATCH) return FA_ERR_NOALLOC_LIMIT;
+  DeviceInfo* info = nullptr;
+  if ((s = device_info(&info)) != FA_OK) return s;
+  void* scratch = nullptr;
+  if ((s = noalloc_scratch(&scratch)) != FA_OK) return s;
+  // The preprocess kernel rewrites every part of the scratch that must start
+  // from zero (dQ accumulator, scheduler counter), so the previous call's
+  // contents do not matter.
+  return launch_bwd(q, k, v, o, dO, lse, dq, dk, dv, B, H, N, d, scale, causal != 0, scratch,
+                    grad_dtype, info->sms, info->status, reinterpret_cast<cudaStream_t>(stream));
 }
 
 }  // extern "C"

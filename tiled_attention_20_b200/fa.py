@@ -22,11 +22,13 @@ STATUS_NAMES = {
     0: "FA_OK", -1: "FA_ERR_NULL", -2: "FA_ERR_SHAPE", -3: "FA_ERR_UNSUPPORTED_D",
     -4: "FA_ERR_ALIGN", -5: "FA_ERR_WORKSPACE", -6: "FA_ERR_LAUNCH", -7: "FA_ERR_TIMEOUT",
     -8: "FA_ERR_DEVICE_ASSERT", -9: "FA_ERR_ARCH", -10: "FA_ERR_ARG",
+    -11: "FA_ERR_NOALLOC_LIMIT",
 }
 
 EXPORTED = ["fa_fwd", "fa_bwd", "fa_bwd_workspace_size", "fa_strerror",
             "fa_check_device_errors", "fa_launch_shape", "fa_trace_start", "fa_trace_stop",
-            "fa_trace_kernel_name"]
+            "fa_trace_kernel_name", "fa_bwd_noalloc"]
+NOALLOC_MAX_SCRATCH = 32 << 20  # FA_BWD_NOALLOC_MAX_SCRATCH
 KERNEL_IDS = {0: "fa_fwd_kernel", 1: "fa_bwd_prep", 2: "fa_bwd_kernel", 3: "fa_bwd_dq_convert"}
 
 
@@ -69,6 +71,9 @@ def load(path: str = LIB_PATH):
         lib.fa_trace_stop.restype = _i
         lib.fa_trace_kernel_name.argtypes = [_i]
         lib.fa_trace_kernel_name.restype = ctypes.c_char_p
+        lib.fa_bwd_noalloc.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp,
+                                       _i, _i, _i, _i, _f, _i, _i, _vp]
+        lib.fa_bwd_noalloc.restype = _i
         _lib = lib
     return _lib
 
@@ -148,6 +153,32 @@ def bwd(q, k, v, o, dO, lse, scale=None, causal=False, grad_dtype=torch.bfloat16
                            dv.data_ptr(), B, H, N, d, scale, int(bool(causal)),
                            workspace.data_ptr(), workspace.numel(), gd, _stream(q.device))
     _check(st, "fa_bwd")
+    return dq, dk, dv
+
+
+def bwd_noalloc(q, k, v, o, dO, lse, scale=None, causal=False, grad_dtype=torch.bfloat16,
+                dq=None, dk=None, dv=None):
+    """fa_bwd_noalloc: the backward with the library's fixed internal scratch
+    instead of a caller workspace, for callers that cannot allocate device
+    memory (the outputs here are still allocated by PyTorch for convenience;
+    such a caller passes its own).  Problems needing more than
+    NOALLOC_MAX_SCRATCH bytes of scratch raise FA_ERR_NOALLOC_LIMIT; calls
+    that overlap on the GPU share the scratch and must not run concurrently."""
+    _check_qkv(q, k, v, o, dO)
+    B, H, N, d = q.shape
+    if lse.dtype != torch.float32 or tuple(lse.shape) != (B, H, N) or not lse.is_contiguous():
+        raise ValueError("lse must be contiguous fp32 [B, H, N]")
+    scale = default_scale(d) if scale is None else float(scale)
+    gd = {torch.bfloat16: 0, torch.float32: 1}[grad_dtype]
+    dq = torch.empty(q.shape, dtype=grad_dtype, device=q.device) if dq is None else dq
+    dk = torch.empty(q.shape, dtype=grad_dtype, device=q.device) if dk is None else dk
+    dv = torch.empty(q.shape, dtype=grad_dtype, device=q.device) if dv is None else dv
+    with torch.cuda.device(q.device):
+        st = load().fa_bwd_noalloc(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(),
+                                   dO.data_ptr(), lse.data_ptr(), dq.data_ptr(), dk.data_ptr(),
+                                   dv.data_ptr(), B, H, N, d, scale, int(bool(causal)), gd,
+                                   _stream(q.device))
+    _check(st, "fa_bwd_noalloc")
     return dq, dk, dv
 
 
