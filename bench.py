@@ -40,7 +40,7 @@ if ROOT not in sys.path:
 
 import torch  # noqa: E402
 
-from tiled_attention_20_b200 import inputs, perf  # noqa: E402
+from tiled_attention_20_b200 import inputs, perf, ranks  # noqa: E402
 
 WORKLOAD = inputs.GPT_CAUSAL
 METRIC = "attention fwd+bwd TFLOP/s (bf16, causal, N=4096 d=128) and % of dense BF16 peak"
@@ -95,18 +95,19 @@ def kernel_source_hash() -> str:
 
 
 def profiled_traffic(kernel: str):
-    """DRAM bytes per launch of `kernel` from the committed ncu summary, if it
-    was captured from the current kernel sources; else None."""
-    path = os.path.join(ROOT, "profiles", "traffic.json")
+    """DRAM bytes per launch of `kernel` from the committed ncu summary
+    (profiles/dram_traffic.txt), if it was captured from the current kernel
+    sources; else None."""
+    path = os.path.join(ROOT, "profiles", "dram_traffic.txt")
     try:
         with open(path) as f:
-            rec = json.load(f)
-    except (OSError, ValueError):
+            lines = [l.split() for l in f if l.strip() and not l.startswith("#")]
+    except OSError:
         return None
-    ent = rec.get(kernel)
-    if not ent or ent.get("source_hash") != kernel_source_hash():
-        return None
-    return ent.get("dram_bytes_per_launch")
+    for name, src_hash, nbytes in (l[:3] for l in lines if len(l) >= 3):
+        if name == kernel and src_hash == kernel_source_hash():
+            return int(nbytes)
+    return None
 
 
 # ---------------------------------------------------------------- clocks
@@ -229,7 +230,8 @@ def run_ours(args, rank, world, local_rank, dist):
     dev = torch.device("cuda", local_rank)
     torch.cuda.set_device(dev)
     w = WORKLOAD
-    q_h, k_h, v_h, dO_h = inputs.qkv_do(w.B, w.H, w.N, w.d, seed=w.seed + rank, dist=w.dist)
+    q_h, k_h, v_h, dO_h = inputs.qkv_do(w.B, w.H, w.N, w.d, seed=ranks.rank_seed(w.seed, rank),
+                                        dist=w.dist)
     q, k, v, dO = (t.to(dev) for t in (q_h, k_h, v_h, dO_h))
     o = torch.empty_like(q)
     lse = torch.empty((w.B, w.H, w.N), dtype=torch.float32, device=dev)
@@ -275,13 +277,9 @@ def run_ours(args, rank, world, local_rank, dist):
         dist.barrier()
     clocks = sampler.stop()
     fa.check_device_errors(dev)
-    ms = e0.elapsed_time(e1) / args.steps
-    if world > 1:
-        t = torch.tensor([ms], device=dev, dtype=torch.float64)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms = float(t.item())
+    ms = ranks.max_over_ranks(e0.elapsed_time(e1) / args.steps, dist, dev)
     flops = step_flops(w)
-    value = flops * world / (ms * 1e-3) / 1e12
+    value = ranks.weak_scaling_rate(flops, world, ms) / 1e12
 
     # dominant kernel by traced time
     dom = max(traced.items(), key=lambda kv: kv[1][1])
@@ -337,13 +335,9 @@ def run_ours(args, rank, world, local_rank, dist):
             e2e_step()
         e1.record(stream)
         torch.cuda.synchronize(dev)
-        ms_e2e = e0.elapsed_time(e1) / n_e2e
-        if world > 1:
-            t = torch.tensor([ms_e2e], device=dev, dtype=torch.float64)
-            dist.all_reduce(t, op=dist.ReduceOp.MAX)
-            ms_e2e = float(t.item())
+        ms_e2e = ranks.max_over_ranks(e0.elapsed_time(e1) / n_e2e, dist, dev)
         nb = lambda *ts: sum(t.numel() * t.element_size() for t in ts)
-        e2e = {"value": flops * world / (ms_e2e * 1e-3) / 1e12, "unit": UNIT,
+        e2e = {"value": ranks.weak_scaling_rate(flops, world, ms_e2e) / 1e12, "unit": UNIT,
                "h2d_bytes_per_step": nb(hq, hk, hv, hdO),
                "d2h_bytes_per_step": nb(ho, hlse, hdq, hdk, hdv), "steps": n_e2e,
                "ms_per_step": ms_e2e, "api": "tiled_attention_20_b200.fa.fwd/bwd (C ABI)"}
@@ -371,9 +365,8 @@ def run_ours(args, rank, world, local_rank, dist):
 
 def main():
     args = parse_args()
-    world = int(os.environ.get("WORLD_SIZE", "1"))
-    rank = int(os.environ.get("RANK", "0"))
-    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    info = ranks.rank_info()
+    world, rank, local_rank = info.world, info.rank, info.local_rank
     if args.impl == "reference":
         run_reference(args, rank, world)
         return
