@@ -165,6 +165,7 @@ __device__ __forceinline__ bool bwait1(uint64_t* bar, uint32_t parity, BwdBarrie
   return false;
 }
 
+// The same from every lane of a warp, with a warp-uniform answer.
 __device__ __forceinline__ bool bwait_warp(uint64_t* bar, uint32_t parity, BwdBarriers* b,
                                            int* status) {
   bool ok = !*(volatile int*)&b->abort_flag;
@@ -475,11 +476,16 @@ __device__ void bwd_compute(const BwdParams& p, uint8_t* smem, BwdBarriers* b, u
         *reinterpret_cast<uint4*>(ds_row + ((piece ^ (t & 7)) << 4)) =
             make_uint4(w4[0], w4[1], w4[2], w4[3]);
       }
+      // Each lane orders its own TMEM and shared-memory writes; after the
+      // warp synchronises, one arrival per warp publishes the warp's work.
       tmem_st_wait();
       tc_fence_before();
-      mbar_arrive(&b->p_ready[s]);
       fence_proxy_async_smem();
-      mbar_arrive(&b->ds_ready[s]);
+      __syncwarp();
+      if (lane_id() == 0) {
+        mbar_arrive(&b->p_ready[s]);
+        mbar_arrive(&b->ds_ready[s]);
+      }
     }
     // Unit epilogue: warpgroup 0 writes dV, warpgroup 1 writes scale * dK.
     if (!bwait_warp(&b->acc_full, uc & 1, b, p.status)) return;
@@ -495,7 +501,8 @@ __device__ void bwd_compute(const BwdParams& p, uint8_t* smem, BwdBarriers* b, u
     else
       tmem_ld_x64(tmem + lane_base + col, r);
     tc_fence_before();
-    mbar_arrive(&b->acc_empty);  // TMEM read: the next unit may overwrite dK, dV
+    __syncwarp();
+    if (lane_id() == 0) mbar_arrive(&b->acc_empty);  // TMEM read: dK, dV may be overwritten
     if (valid) {
       if (p.grad_f32) {
         float4* dst = reinterpret_cast<float4*>(static_cast<float*>(out) + row * D);
@@ -552,7 +559,8 @@ __device__ void bwd_drain(const BwdParams& p, uint8_t* smem, BwdBarriers* b, uin
       uint32_t r[64];
       tmem_ld_x64(tmem + lane_base + L::kTdP + 64 * s, r);
       tc_fence_before();
-      mbar_arrive(&b->dq_empty[s]);
+      __syncwarp();
+      if (lane_id() == 0) mbar_arrive(&b->dq_empty[s]);
 #pragma unroll
       for (int half = 0; half < 2; ++half) {
         float* stage = reinterpret_cast<float*>(smem + L::kStage + half * L::kStageBytes);
@@ -601,13 +609,13 @@ __global__ void __launch_bounds__(512, 1)
     for (int i = 0; i < 2; ++i) {
       mbar_init(&b->s_full[i], 1);
       mbar_init(&b->dp_full[i], 1);
-      mbar_init(&b->p_ready[i], 128);
-      mbar_init(&b->ds_ready[i], 128);
+      mbar_init(&b->p_ready[i], 4);   // one arrival per compute warp
+      mbar_init(&b->ds_ready[i], 4);
       mbar_init(&b->dq_full[i], 1);
-      mbar_init(&b->dq_empty[i], 128);
+      mbar_init(&b->dq_empty[i], 4);  // one arrival per drain warp
     }
     mbar_init(&b->acc_full, 1);
-    mbar_init(&b->acc_empty, 256);
+    mbar_init(&b->acc_empty, 8);  // one arrival per compute warp
     for (int i = 0; i < kUnitRing; ++i) {
       mbar_init(&b->unit_full[i], 1);
       mbar_init(&b->unit_empty[i], kUnitConsumers);

@@ -120,6 +120,7 @@ __device__ __forceinline__ bool wait1(uint64_t* bar, uint32_t parity, FwdBarrier
 }
 
 // The same from every lane of a warp, with a warp-uniform answer.
+// The same from every lane of a warp, with a warp-uniform answer.
 __device__ __forceinline__ bool wait_warp(uint64_t* bar, uint32_t parity, FwdBarriers* b,
                                           int* status) {
   bool ok = !*(volatile int*)&b->abort_flag;
@@ -384,7 +385,8 @@ __device__ void fwd_softmax(const FwdParams& p, FwdBarriers* b, uint32_t tmem, i
       l += rsum.x + rsum.y;
       tmem_st_wait();
       tc_fence_before();
-      mbar_arrive(&b->p_full[wg]);
+      __syncwarp();
+      if (lane_id() == 0) mbar_arrive(&b->p_full[wg]);  // one arrival per warp
     }
     // Epilogue: O = o / l, lse = (m + log2 l) ln 2.
     if (!wait_warp(&b->o_full[wg], oc & 1, b, p.status)) return;
@@ -393,20 +395,20 @@ __device__ void fwd_softmax(const FwdParams& p, FwdBarriers* b, uint32_t tmem, i
     const float inv_l = 1.f / l;
     const bool valid = row < N;
     __nv_bfloat16* orow = p.o + (static_cast<size_t>(u.bh) * N + row) * D;
+    uint32_t o[D];
+    if (D == 128)
+      tmem_ld_x128(tO, o);
+    else
+      tmem_ld_x64(tO, o);
+    if (valid) {
+      uint4* dst = reinterpret_cast<uint4*>(orow);
 #pragma unroll
-    for (int c0 = 0; c0 < D; c0 += 32) {
-      uint32_t o[32];
-      tmem_ld_x32(tO + c0, o);
-      uint32_t pkd[16];
-#pragma unroll
-      for (int c = 0; c < 16; ++c)
-        pkd[c] = pack_bf16x2(__uint_as_float(o[2 * c]) * inv_l, __uint_as_float(o[2 * c + 1]) * inv_l);
-      if (valid) {
-        uint4* dst = reinterpret_cast<uint4*>(orow + c0);
-#pragma unroll
-        for (int v = 0; v < 4; ++v)
-          dst[v] = make_uint4(pkd[4 * v], pkd[4 * v + 1], pkd[4 * v + 2], pkd[4 * v + 3]);
-      }
+      for (int v = 0; v < D / 8; ++v)
+        dst[v] = make_uint4(
+            pack_bf16x2(__uint_as_float(o[8 * v + 0]) * inv_l, __uint_as_float(o[8 * v + 1]) * inv_l),
+            pack_bf16x2(__uint_as_float(o[8 * v + 2]) * inv_l, __uint_as_float(o[8 * v + 3]) * inv_l),
+            pack_bf16x2(__uint_as_float(o[8 * v + 4]) * inv_l, __uint_as_float(o[8 * v + 5]) * inv_l),
+            pack_bf16x2(__uint_as_float(o[8 * v + 6]) * inv_l, __uint_as_float(o[8 * v + 7]) * inv_l));
     }
     if (valid) p.lse[static_cast<size_t>(u.bh) * N + row] = (m_used + __log2f(l)) * 0.69314718055994531f;
   }
@@ -435,7 +437,7 @@ __global__ void __launch_bounds__(384, 1)
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(&b->s_full[i], 1);
-      mbar_init(&b->p_full[i], 128);
+      mbar_init(&b->p_full[i], 4);
       mbar_init(&b->o_full[i], 1);
     }
     mbar_init(&b->mma_done, 1);
