@@ -99,11 +99,31 @@ int fa_bwd(const void *q, const void *k, const void *v, const void *o,
            void *workspace, size_t workspace_bytes, int grad_dtype,
            fa_stream_t stream);
 
-/* Bytes of scratch fa_bwd needs: an fp32 dQ accumulator [B,H,N,d], then
- * lse * log2(e) and D = rowsum(dO * O) as fp32 [B,H,Npad] with Npad = N
- * rounded up to 64, each rounded up to 256 bytes, then 256 bytes for the
- * work-unit counter of the dynamic scheduler.  0 on invalid shapes. */
+/* Bytes of scratch fa_bwd (and fa_bwd_deterministic) needs: an fp32 dQ
+ * accumulator [B,H,N,d], then lse * log2(e) and D = rowsum(dO * O) as fp32
+ * [B,H,Npad] with Npad = N rounded up to 128, each rounded up to 256 bytes,
+ * then 256 bytes for the work-unit counter of the dynamic scheduler.
+ * 0 on invalid shapes. */
 size_t fa_bwd_workspace_size(int B, int H, int N, int d);
+
+/*
+ * Deterministic backward: the same gradients, arguments, layouts, workspace
+ * and errors as fa_bwd, but every output bit is reproducible from run to run.
+ * fa_bwd sums the per-block dQ contributions with fp32 reduce-add copies in
+ * an order that varies; here dK and dV come from the same key-block-major
+ * kernel without its dQ part, and a second, query-block-major kernel
+ * recomputes P and dS tile by tile in a fixed key order and writes each dQ
+ * row once.  It does three more tile multiplications per tile pair than
+ * fa_bwd (S and dP are formed twice) but sends no dQ traffic through L2
+ * reductions.  Not on the pages, whose only statement on the subject is that
+ * tiled attention is not bit-identical to the untiled computation (§8.4 of
+ * the first page).
+ */
+int fa_bwd_deterministic(const void *q, const void *k, const void *v, const void *o,
+                         const void *dO, const float *lse, void *dq, void *dk, void *dv,
+                         int B, int H, int N, int d, float scale, int causal,
+                         void *workspace, size_t workspace_bytes, int grad_dtype,
+                         fa_stream_t stream);
 
 /* Human-readable text for an fa_status value (static storage). */
 const char *fa_strerror(int status);
@@ -128,7 +148,8 @@ int fa_launch_shape(int pass, int B, int H, int N, int d, int causal,
  * until fa_trace_stop().  fa_trace_stop() waits for those events and fills,
  * for each kernel id k < n_kernels, launches[k] and total_ms[k] (summed event
  * durations).  Kernel ids: 0 forward, 1 backward preprocess, 2 backward main,
- * 3 dQ conversion (fa_trace_kernel_name gives the kernel's name).  The
+ * 3 dQ conversion, 4 dQ pass of the deterministic backward
+ * (fa_trace_kernel_name gives the kernel's name).  The
  * library creates the events on first use and reuses them afterwards; event
  * records add a few microseconds per launch.  fa_trace_start() discards a
  * previous unfinished record.

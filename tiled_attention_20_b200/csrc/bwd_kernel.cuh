@@ -51,9 +51,10 @@ inline int bwd_units(int B, int H, int N) { return B * H * ((N + 127) / 128); }
 inline size_t round256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
 
 // Workspace: dQ accumulator [BH][N][d] fp32, then lse*log2e and D, each
-// [BH][Npad] fp32 with Npad = N rounded up to 64, then the scheduler's
+// [BH][Npad] fp32 with Npad = N rounded up to 128 (whole 64-row and 128-row
+// query blocks read padding, never the next head), then the scheduler's
 // work-unit counter.
-inline size_t bwd_npad(int N) { return (static_cast<size_t>(N) + 63) / 64 * 64; }
+inline size_t bwd_npad(int N) { return (static_cast<size_t>(N) + 127) / 128 * 128; }
 inline size_t bwd_workspace_bytes(int B, int H, int N, int d) {
   const size_t bh = static_cast<size_t>(B) * H;
   return round256(bh * N * d * 4) + 2 * round256(bh * bwd_npad(N) * 4) + 256;
@@ -121,8 +122,9 @@ static_assert(128 * kBwdCtlRegs + 256 * kBwdComputeRegs + 128 * kBwdDrainRegs <=
 
 constexpr int kUnitRing = 4;
 // Consumers of the unit ring, counted in arrivals: the MMA thread, the 8
-// compute warps and the 4 drain warps (one lane each).
-constexpr int kUnitConsumers = 1 + 8 + 4;
+// compute warps and, when the kernel computes dQ, the 4 drain warps (one
+// lane each).
+constexpr int unit_consumers(bool dq) { return 1 + 8 + (dq ? 4 : 0); }
 
 struct BwdBarriers {
   uint64_t kv_full, kv_empty;
@@ -337,7 +339,7 @@ struct BwdMma {
   }
 };
 
-template <int D, bool CAUSAL>
+template <int D, bool CAUSAL, bool DQ>
 __device__ void bwd_mma(const BwdParams& p, uint8_t* smem, BwdBarriers* b, uint32_t tmem) {
   using L = BwdLayout<D>;
   using M = BwdMma<D>;
@@ -358,7 +360,7 @@ __device__ void bwd_mma(const BwdParams& p, uint8_t* smem, BwdBarriers* b, uint3
       tc_fence_after();
       M::kq(tmem + L::kTS + 64 * s, sb + L::kK, sb + L::kQ + qs * L::kQBytes);
       mma_commit(&b->s_full[s]);
-      if (gg >= 2) {
+      if (DQ && gg >= 2) {
         if (!bwait1(&b->dq_empty[s], ((gg >> 1) - 1) & 1, b, p.status)) return false;
         tc_fence_after();
       }
@@ -378,8 +380,10 @@ __device__ void bwd_mma(const BwdParams& p, uint8_t* smem, BwdBarriers* b, uint3
       if (!bwait1(&b->ds_ready[s], (gg >> 1) & 1, b, p.status)) return false;
       tc_fence_after();
       M::dk(tmem + L::kTdK, sb + L::kDs + s * L::kDsBytes, sb + L::kQ + qs * L::kQBytes, it > 0);
-      M::dqt(tmem + L::kTdP + 64 * s, sb + L::kK, sb + L::kDs + s * L::kDsBytes);
-      mma_commit(&b->dq_full[s]);
+      if (DQ) {
+        M::dqt(tmem + L::kTdP + 64 * s, sb + L::kK, sb + L::kDs + s * L::kDsBytes);
+        mma_commit(&b->dq_full[s]);
+      }
       mma_commit(&b->q_empty[qs]);
       return true;
     };
@@ -588,7 +592,9 @@ __device__ void bwd_drain(const BwdParams& p, uint8_t* smem, BwdBarriers* b, uin
 }
 
 // ---------------------------------------------------------------- kernels
-template <int D, bool CAUSAL>
+// DQ = false computes dK and dV only (the deterministic backward computes dQ
+// in a separate pass, fa_dq_kernel).
+template <int D, bool CAUSAL, bool DQ>
 __global__ void __launch_bounds__(512, 1)
     fa_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                   const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
@@ -618,7 +624,7 @@ __global__ void __launch_bounds__(512, 1)
     mbar_init(&b->acc_empty, 8);  // one arrival per compute warp
     for (int i = 0; i < kUnitRing; ++i) {
       mbar_init(&b->unit_full[i], 1);
-      mbar_init(&b->unit_empty[i], kUnitConsumers);
+      mbar_init(&b->unit_empty[i], unit_consumers(DQ));
     }
     mbar_init(&b->mma_done, 1);
     b->abort_flag = 0;
@@ -644,7 +650,7 @@ __global__ void __launch_bounds__(512, 1)
     bwd_compute<D, CAUSAL>(p, smem, b, tmem, (warp - 4) >> 2);
   } else if (warp >= 12) {
     regs_decrease<kBwdDrainRegs>();
-    bwd_drain<D, CAUSAL>(p, smem, b, tmem);
+    if (DQ) bwd_drain<D, CAUSAL>(p, smem, b, tmem);
   } else {
     regs_decrease<kBwdCtlRegs>();
     if (warp == 0) {
@@ -662,7 +668,7 @@ __global__ void __launch_bounds__(512, 1)
       __syncwarp();
     } else if (warp == 1) {
       if (lane_id() == 0) {
-        bwd_mma<D, CAUSAL>(p, smem, b, tmem);
+        bwd_mma<D, CAUSAL, DQ>(p, smem, b, tmem);
         mma_commit(&b->mma_done);
         mbar_wait(&b->mma_done, 0, p.status);
       }
@@ -681,7 +687,8 @@ template <int D>
 __global__ void __launch_bounds__(256)
     fa_bwd_prep(const __nv_bfloat16* __restrict__ o, const __nv_bfloat16* __restrict__ dO,
                 const float* __restrict__ lse, float* __restrict__ lse2, float* __restrict__ dvec,
-                float* __restrict__ dq_acc, int* __restrict__ sched, int BH, int N, int Npad) {
+                float* __restrict__ dq_acc, int* __restrict__ sched, int BH, int N, int Npad,
+                int zero_acc) {
   constexpr int TPR = D / 8;  // threads per row
   if (blockIdx.x == 0 && threadIdx.x == 0) *sched = 0;
   const long long gid = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x;
@@ -705,9 +712,11 @@ __global__ void __launch_bounds__(256)
       acc = fmaf(x.x, y.x, acc);
       acc = fmaf(x.y, y.y, acc);
     }
-    float4* z = reinterpret_cast<float4*>(dq_acc + off);
-    z[0] = make_float4(0.f, 0.f, 0.f, 0.f);
-    z[1] = make_float4(0.f, 0.f, 0.f, 0.f);
+    if (zero_acc) {
+      float4* z = reinterpret_cast<float4*>(dq_acc + off);
+      z[0] = make_float4(0.f, 0.f, 0.f, 0.f);
+      z[1] = make_float4(0.f, 0.f, 0.f, 0.f);
+    }
   }
 #pragma unroll
   for (int m = TPR / 2; m >= 1; m >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, m, TPR);

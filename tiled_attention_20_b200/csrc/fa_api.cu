@@ -14,6 +14,7 @@
 
 #include "../../include/fa.h"
 #include "bwd_kernel.cuh"
+#include "dq_kernel.cuh"
 #include "fwd_kernel.cuh"
 
 namespace {
@@ -43,9 +44,10 @@ EncodeTiledFn g_encode = nullptr;
 // ---------------------------------------------------------------- tracing
 // Opt-in per-kernel timing: while enabled, every launch is bracketed by a
 // pair of CUDA events on its stream.
-enum { kKernFwd = 0, kKernBwdPrep = 1, kKernBwd = 2, kKernBwdConvert = 3, kNumKernels = 4 };
+enum { kKernFwd = 0, kKernBwdPrep = 1, kKernBwd = 2, kKernBwdConvert = 3, kKernDq = 4,
+       kNumKernels = 5 };
 const char* const kKernelNames[kNumKernels] = {"fa_fwd_kernel", "fa_bwd_prep", "fa_bwd_kernel",
-                                               "fa_bwd_dq_convert"};
+                                               "fa_bwd_dq_convert", "fa_dq_kernel"};
 struct TraceRec {
   int kernel;
   int device;
@@ -175,11 +177,11 @@ int make_tmap_rows(CUtensorMap* m, const void* base, int BH, int N, int d, int b
   return r == CUDA_SUCCESS ? FA_OK : FA_ERR_LAUNCH;
 }
 
-template <int D, bool CAUSAL>
+template <int D, bool CAUSAL, bool DQ>
 int launch_bwd_main(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                     const CUtensorMap& tdo, const fa::BwdParams& p, int ctas,
                     cudaStream_t stream) {
-  auto kern = fa::fa_bwd_kernel<D, CAUSAL>;
+  auto kern = fa::fa_bwd_kernel<D, CAUSAL, DQ>;
   const int smem = fa::BwdLayout<D>::kSmemBytes;
   // The register split between warpgroups assumes this launch allocation.
   cudaFuncAttributes attr;
@@ -192,10 +194,28 @@ int launch_bwd_main(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensor
   return cudaPeekAtLastError() == cudaSuccess ? FA_OK : FA_ERR_LAUNCH;
 }
 
+template <int D, bool CAUSAL>
+int launch_dq(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
+              const CUtensorMap& tdo, const fa::DqParams& p, int ctas, cudaStream_t stream) {
+  auto kern = fa::fa_dq_kernel<D, CAUSAL>;
+  const int smem = fa::DqLayout<D>::kSmemBytes;
+  cudaFuncAttributes attr;
+  if (cudaFuncGetAttributes(&attr, kern) != cudaSuccess || attr.numRegs != fa::kDqLaunchRegs)
+    return FA_ERR_LAUNCH;
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
+    return FA_ERR_LAUNCH;
+  LaunchTrace trace(kKernDq, stream);
+  kern<<<ctas, 384, smem, stream>>>(tq, tk, tv, tdo, p);
+  return cudaPeekAtLastError() == cudaSuccess ? FA_OK : FA_ERR_LAUNCH;
+}
+
+// Backward: preprocess, then either the atomic main kernel (dQ, dK, dV) and
+// the dQ conversion, or (deterministic) the main kernel without dQ and the
+// query-block-major dQ kernel.
 int launch_bwd(const void* q, const void* k, const void* v, const void* o, const void* dO,
                const float* lse, void* dq, void* dk, void* dv, int B, int H, int N, int d,
                float scale, bool causal, void* workspace, int grad_dtype, int sms, int* status,
-               cudaStream_t stream) {
+               cudaStream_t stream, bool deterministic = false) {
   const int BH = B * H;
   const size_t npad = fa::bwd_npad(N);
   uint8_t* ws = static_cast<uint8_t*>(workspace);
@@ -217,11 +237,11 @@ int launch_bwd(const void* q, const void* k, const void* v, const void* o, const
     if (d == 64)
       fa::fa_bwd_prep<64><<<blocks, 256, 0, stream>>>(
           static_cast<const __nv_bfloat16*>(o), static_cast<const __nv_bfloat16*>(dO), lse, lse2,
-          dvec, dq_acc, sched, BH, N, static_cast<int>(npad));
+          dvec, dq_acc, sched, BH, N, static_cast<int>(npad), deterministic ? 0 : 1);
     else
       fa::fa_bwd_prep<128><<<blocks, 256, 0, stream>>>(
           static_cast<const __nv_bfloat16*>(o), static_cast<const __nv_bfloat16*>(dO), lse, lse2,
-          dvec, dq_acc, sched, BH, N, static_cast<int>(npad));
+          dvec, dq_acc, sched, BH, N, static_cast<int>(npad), deterministic ? 0 : 1);
     if (cudaPeekAtLastError() != cudaSuccess) return FA_ERR_LAUNCH;
   }
   // 2. tensor-core main kernel
@@ -244,12 +264,44 @@ int launch_bwd(const void* q, const void* k, const void* v, const void* o, const
   p.status = status;
   const int ctas = p.n_units < sms ? p.n_units : sms;
   int rc;
+  if (deterministic) {
+    if (d == 64)
+      rc = causal ? launch_bwd_main<64, true, false>(tq, tk, tv, tdo, p, ctas, stream)
+                  : launch_bwd_main<64, false, false>(tq, tk, tv, tdo, p, ctas, stream);
+    else
+      rc = causal ? launch_bwd_main<128, true, false>(tq, tk, tv, tdo, p, ctas, stream)
+                  : launch_bwd_main<128, false, false>(tq, tk, tv, tdo, p, ctas, stream);
+    if (rc != FA_OK) return rc;
+    CUtensorMap tq128, tdo128;
+    if (make_tmap_rows(&tq128, q, BH, N, d, 128) != FA_OK ||
+        make_tmap_rows(&tdo128, dO, BH, N, d, 128) != FA_OK)
+      return FA_ERR_LAUNCH;
+    fa::DqParams dp;
+    dp.dq = dq;
+    dp.lse2 = lse2;
+    dp.dvec = dvec;
+    dp.BH = BH;
+    dp.N = N;
+    dp.Npad = static_cast<int>(npad);
+    dp.nqt = (N + 127) / 128;
+    dp.n_units = BH * dp.nqt;
+    dp.scale_log2 = scale * 1.4426950408889634f;
+    dp.scale = scale;
+    dp.grad_f32 = grad_dtype;
+    dp.status = status;
+    const int dctas = dp.n_units < sms ? dp.n_units : sms;
+    if (d == 64)
+      return causal ? launch_dq<64, true>(tq128, tk, tv, tdo128, dp, dctas, stream)
+                    : launch_dq<64, false>(tq128, tk, tv, tdo128, dp, dctas, stream);
+    return causal ? launch_dq<128, true>(tq128, tk, tv, tdo128, dp, dctas, stream)
+                  : launch_dq<128, false>(tq128, tk, tv, tdo128, dp, dctas, stream);
+  }
   if (d == 64)
-    rc = causal ? launch_bwd_main<64, true>(tq, tk, tv, tdo, p, ctas, stream)
-                : launch_bwd_main<64, false>(tq, tk, tv, tdo, p, ctas, stream);
+    rc = causal ? launch_bwd_main<64, true, true>(tq, tk, tv, tdo, p, ctas, stream)
+                : launch_bwd_main<64, false, true>(tq, tk, tv, tdo, p, ctas, stream);
   else
-    rc = causal ? launch_bwd_main<128, true>(tq, tk, tv, tdo, p, ctas, stream)
-                : launch_bwd_main<128, false>(tq, tk, tv, tdo, p, ctas, stream);
+    rc = causal ? launch_bwd_main<128, true, true>(tq, tk, tv, tdo, p, ctas, stream)
+                : launch_bwd_main<128, false, true>(tq, tk, tv, tdo, p, ctas, stream);
   if (rc != FA_OK) return rc;
   // 3. dQ = scale * accumulator
   {
@@ -361,6 +413,26 @@ int fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int
                   : launch_fwd<64, false>(tq, tk, tv, p, ctas, st);
   return causal ? launch_fwd<128, true>(tq, tk, tv, p, ctas, st)
                 : launch_fwd<128, false>(tq, tk, tv, p, ctas, st);
+}
+
+int fa_bwd_deterministic(const void* q, const void* k, const void* v, const void* o,
+                         const void* dO, const float* lse, void* dq, void* dk, void* dv, int B,
+                         int H, int N, int d, float scale, int causal, void* workspace,
+                         size_t workspace_bytes, int grad_dtype, fa_stream_t stream) {
+  if (!q || !k || !v || !o || !dO || !lse || !dq || !dk || !dv || !workspace) return FA_ERR_NULL;
+  int s = check_shape(B, H, N, d);
+  if (s != FA_OK) return s;
+  if ((s = check_scale(scale)) != FA_OK) return s;
+  if (grad_dtype != 0 && grad_dtype != 1) return FA_ERR_ARG;
+  const void* ptrs[] = {q, k, v, o, dO, lse, dq, dk, dv, workspace};
+  for (const void* ptr : ptrs)
+    if (!aligned16(ptr)) return FA_ERR_ALIGN;
+  if (workspace_bytes < fa::bwd_workspace_bytes(B, H, N, d)) return FA_ERR_WORKSPACE;
+  DeviceInfo* info = nullptr;
+  if ((s = device_info(&info)) != FA_OK) return s;
+  return launch_bwd(q, k, v, o, dO, lse, dq, dk, dv, B, H, N, d, scale, causal != 0, workspace,
+                    grad_dtype, info->sms, info->status, reinterpret_cast<cudaStream_t>(stream),
+                    true);
 }
 
 size_t fa_bwd_workspace_size(int B, int H, int N, int d) {

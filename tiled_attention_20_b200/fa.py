@@ -27,9 +27,10 @@ STATUS_NAMES = {
 
 EXPORTED = ["fa_fwd", "fa_bwd", "fa_bwd_workspace_size", "fa_strerror",
             "fa_check_device_errors", "fa_launch_shape", "fa_trace_start", "fa_trace_stop",
-            "fa_trace_kernel_name", "fa_bwd_noalloc"]
+            "fa_trace_kernel_name", "fa_bwd_noalloc", "fa_bwd_deterministic"]
 NOALLOC_MAX_SCRATCH = 32 << 20  # FA_BWD_NOALLOC_MAX_SCRATCH
-KERNEL_IDS = {0: "fa_fwd_kernel", 1: "fa_bwd_prep", 2: "fa_bwd_kernel", 3: "fa_bwd_dq_convert"}
+KERNEL_IDS = {0: "fa_fwd_kernel", 1: "fa_bwd_prep", 2: "fa_bwd_kernel", 3: "fa_bwd_dq_convert",
+              4: "fa_dq_kernel"}
 
 
 class FAError(RuntimeError):
@@ -56,6 +57,8 @@ def load(path: str = LIB_PATH):
         lib.fa_bwd.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp,
                                _i, _i, _i, _i, _f, _i, _vp, _sz, _i, _vp]
         lib.fa_bwd.restype = _i
+        lib.fa_bwd_deterministic.argtypes = lib.fa_bwd.argtypes
+        lib.fa_bwd_deterministic.restype = _i
         lib.fa_bwd_workspace_size.argtypes = [_i, _i, _i, _i]
         lib.fa_bwd_workspace_size.restype = _sz
         lib.fa_strerror.argtypes = [_i]
@@ -133,8 +136,9 @@ def workspace_size(B, H, N, d) -> int:
 
 
 def bwd(q, k, v, o, dO, lse, scale=None, causal=False, grad_dtype=torch.bfloat16,
-        workspace=None, dq=None, dk=None, dv=None):
-    """dQ, dK, dV [B,H,N,d] (bf16 or fp32) for the forward that produced o, lse."""
+        workspace=None, dq=None, dk=None, dv=None, deterministic=False):
+    """dQ, dK, dV [B,H,N,d] (bf16 or fp32) for the forward that produced o, lse.
+    deterministic=True calls fa_bwd_deterministic (bit-reproducible dQ)."""
     _check_qkv(q, k, v, o, dO)
     B, H, N, d = q.shape
     if lse.dtype != torch.float32 or tuple(lse.shape) != (B, H, N) or not lse.is_contiguous():
@@ -148,11 +152,12 @@ def bwd(q, k, v, o, dO, lse, scale=None, causal=False, grad_dtype=torch.bfloat16
     dk = torch.empty(q.shape, dtype=grad_dtype, device=q.device) if dk is None else dk
     dv = torch.empty(q.shape, dtype=grad_dtype, device=q.device) if dv is None else dv
     with torch.cuda.device(q.device):
-        st = load().fa_bwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(),
-                           dO.data_ptr(), lse.data_ptr(), dq.data_ptr(), dk.data_ptr(),
-                           dv.data_ptr(), B, H, N, d, scale, int(bool(causal)),
-                           workspace.data_ptr(), workspace.numel(), gd, _stream(q.device))
-    _check(st, "fa_bwd")
+        fn = load().fa_bwd_deterministic if deterministic else load().fa_bwd
+        st = fn(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(),
+                dO.data_ptr(), lse.data_ptr(), dq.data_ptr(), dk.data_ptr(),
+                dv.data_ptr(), B, H, N, d, scale, int(bool(causal)),
+                workspace.data_ptr(), workspace.numel(), gd, _stream(q.device))
+    _check(st, "fa_bwd_deterministic" if deterministic else "fa_bwd")
     return dq, dk, dv
 
 
