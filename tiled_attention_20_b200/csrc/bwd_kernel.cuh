@@ -25,8 +25,8 @@
 //               through a 4-entry ring in shared memory; loads K_j, V_j once
 //               per unit and Q_i, dO_i, lse_i, D_i per Q block (3-slot ring).
 //   warp 1      TMEM allocator and single-thread tcgen05.mma issuer.
-//   warps 4-7   compute warpgroup 0, warps 8-11 compute warpgroup 1: they
-//               take alternate Q blocks (pipeline slot s = 0 / 1), one thread
+//   warps 4-7   compute warpgroup 0, warps 8-11 compute warpgroup 1: both
+//               work on every Q block, 32 of its 64 queries each, one thread
 //               per key row: P^T from S^T and lse, dS^T = P^T (dP^T - D).
 //               P^T goes back to TMEM (A of dV += P^T dO), dS^T to shared
 //               memory (A of dK += dS^T Q and, read transposed, B of
@@ -310,14 +310,16 @@ struct BwdMma {
              kk > 0 ? 1u : 0u);
     }
   }
-  // dV += P^T dO (A = P^T from TMEM): M=128 keys, N=D, K=64 queries.
+  // dV += P^T dO (A = P^T from TMEM): M=128 keys, N=D, K=64 queries.  P^T of
+  // queries 0-31 sits in columns [0,16) of the S^T slot, queries 32-63 in
+  // [32,48) (each compute warpgroup writes inside the columns it read).
   static __device__ __forceinline__ void dv(uint32_t d_tmem, uint32_t a_tmem, uint32_t b_do,
                                             bool acc) {
     constexpr uint32_t idesc = idesc_bf16_f32(128, D, false, true);
 #pragma unroll
     for (int kk = 0; kk < 4; ++kk)
-      mma_ts(d_tmem, a_tmem + kk * 8, sdesc_sw128(b_do + kk * 2048, 8192, 1024), idesc,
-             (acc || kk > 0) ? 1u : 0u);
+      mma_ts(d_tmem, a_tmem + 32 * (kk >> 1) + (kk & 1) * 8,
+             sdesc_sw128(b_do + kk * 2048, 8192, 1024), idesc, (acc || kk > 0) ? 1u : 0u);
   }
   // dK += dS^T Q (A = dS^T, K-major in smem): M=128 keys, N=D, K=64 queries.
   static __device__ __forceinline__ void dk(uint32_t d_tmem, uint32_t a_ds, uint32_t b_q,
@@ -401,17 +403,17 @@ __device__ void bwd_mma(const BwdParams& p, uint8_t* smem, BwdBarriers* b, uint3
 }
 
 // ---------------------------------------------------------------- compute warpgroups
+// Both warpgroups work on every Q block: warpgroup h takes queries
+// [32h, 32h+32) of the 64 (thread = key row), so one Q block's element-wise
+// work finishes in half the time.
 template <int D, bool CAUSAL>
 __device__ void bwd_compute(const BwdParams& p, uint8_t* smem, BwdBarriers* b, uint32_t tmem,
-                            int s) {
+                            int h) {
   using L = BwdLayout<D>;
   constexpr int QS = L::kQStages;
   const int t = (threadIdx.x - 128) & 127;  // key row within the K/V block == TMEM lane
   const uint32_t lane_base = static_cast<uint32_t>(t & ~31) << 16;
   const float sl2 = p.scale_log2;
-  const uint32_t tS = tmem + lane_base + L::kTS + 64 * s;
-  const uint32_t tdP = tmem + lane_base + L::kTdP + 64 * s;
-  uint8_t* ds_row = smem + L::kDs + s * L::kDsBytes + t * 128;
   int g = 0, qbase = 0, rc = 0;
   for (int uc = 0;; ++uc) {
     const int w = next_unit_warp(b, rc, p.status);
@@ -419,25 +421,26 @@ __device__ void bwd_compute(const BwdParams& p, uint8_t* smem, BwdBarriers* b, u
     const BwdUnit u = bwd_decode<CAUSAL>(p, w);
     const int key = u.j * 128 + t;
     for (int it = 0; it < u.n; ++it) {
-      const int gg = g + it;
-      if ((gg & 1) != s) continue;
-      const int qs = (qbase + it) % QS;
-      const int q0 = (u.i0 + it) * 64;
+      const int gg = g + it, s = gg & 1, qs = (qbase + it) % QS;
+      const int q0 = (u.i0 + it) * 64 + 32 * h;  // first query of this warpgroup's half
       if (!bwait_warp(&b->s_full[s], (gg >> 1) & 1, b, p.status)) return;
       if (!bwait_warp(&b->dp_full[s], (gg >> 1) & 1, b, p.status)) return;
       tc_fence_after();
-      const float4* lse4 = reinterpret_cast<const float4*>(smem + L::kLse + qs * 256);
-      const float4* dv4 = reinterpret_cast<const float4*>(smem + L::kDv + qs * 256);
+      const uint32_t tS = tmem + lane_base + L::kTS + 64 * s + 32 * h;
+      const uint32_t tdP = tmem + lane_base + L::kTdP + 64 * s + 32 * h;
+      const float4* lse4 = reinterpret_cast<const float4*>(smem + L::kLse + qs * 256) + 8 * h;
+      const float4* dv4 = reinterpret_cast<const float4*>(smem + L::kDv + qs * 256) + 8 * h;
+      uint8_t* ds_row = smem + L::kDs + s * L::kDsBytes + t * 128;
       const bool diag = CAUSAL && q0 < u.j * 128 + 127;
-      uint32_t rs[64], rp[64];
-      tmem_ld_x64_pair(tS, tdP, rs, rp);
+      uint32_t rs[32], rp[32];
+      tmem_ld_x32_pair(tS, tdP, rs, rp);
       const float2 sl2v = make_float2(sl2, sl2);
-      // P^T = exp2(scale*log2e * S^T - lse*log2e), stored to TMEM as bf16
-      // pairs; rs[] keeps P in fp32 for dS.
+      // P^T = exp2(scale*log2e * S^T - lse*log2e) into TMEM as bf16 pairs (the
+      // first 16 of the 32 columns this warpgroup read); rs[] keeps P in fp32.
       {
-        uint32_t pk[32];
+        uint32_t pk[16];
 #pragma unroll
-        for (int c4 = 0; c4 < 16; ++c4) {
+        for (int c4 = 0; c4 < 8; ++c4) {
           const float4 l4 = lse4[c4];
           const int c = 4 * c4;
           const float2 x0 = fma2(make_float2(__uint_as_float(rs[c]), __uint_as_float(rs[c + 1])),
@@ -459,12 +462,12 @@ __device__ void bwd_compute(const BwdParams& p, uint8_t* smem, BwdBarriers* b, u
           pk[2 * c4] = pack_bf16x2(p0, p1);
           pk[2 * c4 + 1] = pack_bf16x2(p2, p3);
         }
-        tmem_st_x32(tS, pk);
+        tmem_st_x16(tS, pk);
       }
       // dS^T = P^T (dP^T - D), to shared memory as bf16 in the 128-byte
-      // swizzled layout the tensor core reads.
+      // swizzled layout the tensor core reads (this half: pieces 4h .. 4h+3).
 #pragma unroll
-      for (int piece = 0; piece < 8; ++piece) {  // 8 queries = 16 bytes per piece
+      for (int piece = 0; piece < 4; ++piece) {  // 8 queries = 16 bytes per piece
         const float4 da = dv4[2 * piece], db = dv4[2 * piece + 1];
         const int c = 8 * piece;
         uint32_t w4[4];
@@ -477,7 +480,8 @@ __device__ void bwd_compute(const BwdParams& p, uint8_t* smem, BwdBarriers* b, u
           const float2 ds = mul2(pp, add2(dp, make_float2(-d2[e].x, -d2[e].y)));
           w4[e] = pack_bf16x2(ds.x, ds.y);
         }
-        *reinterpret_cast<uint4*>(ds_row + ((piece ^ (t & 7)) << 4)) =
+        const int pc = 4 * h + piece;
+        *reinterpret_cast<uint4*>(ds_row + ((pc ^ (t & 7)) << 4)) =
             make_uint4(w4[0], w4[1], w4[2], w4[3]);
       }
       // Each lane orders its own TMEM and shared-memory writes; after the
@@ -496,9 +500,9 @@ __device__ void bwd_compute(const BwdParams& p, uint8_t* smem, BwdBarriers* b, u
     tc_fence_after();
     const bool valid = key < p.N;
     const size_t row = static_cast<size_t>(u.bh) * p.N + key;
-    const uint32_t col = s ? L::kTdK : L::kTdV;
-    const float mul = s ? p.scale : 1.f;
-    void* out = s ? p.dk : p.dv;
+    const uint32_t col = h ? L::kTdK : L::kTdV;
+    const float mul = h ? p.scale : 1.f;
+    void* out = h ? p.dk : p.dv;
     uint32_t r[D];
     if (D == 128)
       tmem_ld_x128(tmem + lane_base + col, r);
@@ -615,8 +619,8 @@ __global__ void __launch_bounds__(512, 1)
     for (int i = 0; i < 2; ++i) {
       mbar_init(&b->s_full[i], 1);
       mbar_init(&b->dp_full[i], 1);
-      mbar_init(&b->p_ready[i], 4);   // one arrival per compute warp
-      mbar_init(&b->ds_ready[i], 4);
+      mbar_init(&b->p_ready[i], 8);   // one arrival per compute warp (both warpgroups)
+      mbar_init(&b->ds_ready[i], 8);
       mbar_init(&b->dq_full[i], 1);
       mbar_init(&b->dq_empty[i], 4);  // one arrival per drain warp
     }
