@@ -45,7 +45,7 @@ from tiled_attention_20_b200 import inputs, perf, ranks  # noqa: E402
 WORKLOAD = inputs.GPT_CAUSAL
 METRIC = "attention fwd+bwd TFLOP/s (bf16, causal, N=4096 d=128) and % of dense BF16 peak"
 UNIT = "TFLOP/s"
-KERNEL_SOURCES = ["fwd_kernel.cuh", "bwd_kernel.cuh", "sm100.cuh", "fa_api.cu"]
+KERNEL_SOURCES = ["fwd_kernel.cuh", "bwd_kernel.cuh", "dq_kernel.cuh", "sm100.cuh", "fa_api.cu"]
 
 
 def parse_args():
@@ -60,6 +60,8 @@ def parse_args():
     ap.add_argument("--no-cpu-baseline", action="store_true",
                     help="skip the CPU oracle leg (used for profiler runs)")
     ap.add_argument("--no-e2e", action="store_true", help="skip the host-buffer leg (profiler runs)")
+    ap.add_argument("--deterministic", action="store_true",
+                    help="time fa_bwd_deterministic (bit-reproducible dQ) instead of fa_bwd")
     return ap.parse_args()
 
 
@@ -240,7 +242,8 @@ def run_ours(args, rank, world, local_rank, dist):
 
     def step():
         fa.fwd(q, k, v, causal=w.causal, out=o, lse=lse)
-        fa.bwd(q, k, v, o, dO, lse, causal=w.causal, workspace=ws, dq=dq, dk=dk, dv=dv)
+        fa.bwd(q, k, v, o, dO, lse, causal=w.causal, workspace=ws, dq=dq, dk=dk, dv=dv,
+               deterministic=args.deterministic)
 
     # Output check before timing (no oracle here): finite results, and row 0
     # of a causal head sees only key 0, so O_0 must equal V_0 bit for bit.
@@ -285,16 +288,23 @@ def run_ours(args, rank, world, local_rank, dist):
     dom = max(traced.items(), key=lambda kv: kv[1][1])
     dom_name, (dom_launches, dom_ms) = dom
     per_launch_ms = dom_ms / dom_launches
+    fwd_f = perf.attention_flops(w.B, w.H, w.N, w.d, w.causal, False)
     kernel_flops = {
-        "fa_fwd_kernel": perf.attention_flops(w.B, w.H, w.N, w.d, w.causal, False),
+        "fa_fwd_kernel": fwd_f,
         "fa_bwd_kernel": perf.attention_flops(w.B, w.H, w.N, w.d, w.causal, True),
     }
+    if args.deterministic:
+        # dK/dV kernel: S, dP, dV, dK (four GEMMs); dQ kernel: S, dP, dQ (three)
+        kernel_flops["fa_bwd_kernel"] = 2.0 * fwd_f
+        kernel_flops["fa_dq_kernel"] = 1.5 * fwd_f
     peaks, peaks_src = measured_peaks()
     if dom_name in kernel_flops:
         achieved = kernel_flops[dom_name] / (per_launch_ms * 1e-3) / 1e12
         roof = {"bound": "tensor", "achieved": achieved, "peak": peaks["bf16_tflops"],
                 "unit": "TFLOP/s", "frac": achieved / peaks["bf16_tflops"],
-                "traffic": profiled_traffic(dom_name), "kernel": dom_name,
+                "traffic": profiled_traffic(dom_name + ("_nodq" if args.deterministic
+                                                             and dom_name == "fa_bwd_kernel" else "")),
+                "kernel": dom_name,
                 "peak_source": f"{peaks_src} bf16_tflops (burst)",
                 "frac_of_sustained": achieved / peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"]),
                 "launch_ms": per_launch_ms}
@@ -355,7 +365,8 @@ def run_ours(args, rank, world, local_rank, dist):
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
             "dtype": "bf16", "data": "synthetic",
-            "config": workload_config(w, {"parallelism": f"heads replicated per GPU x{world}"}),
+            "config": workload_config(w, {"parallelism": f"heads replicated per GPU x{world}",
+                                          "bwd": "deterministic" if args.deterministic else "atomic_dq"}),
             "pct_of_peak": value / world / peaks["bf16_tflops"],
             "roofline": roof, "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": gpu_launches,
             "kernels": kernels, "clocks": clocks,
