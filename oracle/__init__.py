@@ -14,7 +14,10 @@ are stated in the C file's header:
   ("第17讲 Tensor Core、HBM、SRAM 与 FlashAttention", §8.1 and §8.3);
 * lse = m + ln l per row (natural log of the scaled scores);
 * backward: the exact gradient of sum(O * dO) (pages silent; calculus);
-* ``online_fwd``: the online-softmax recurrence of the same page's §8.3.
+* ``online_fwd``: the online-softmax recurrence of the same page's §8.3;
+* ``decode``: the same attention for a few new queries against a key/value
+  cache (the same page's §9.2–9.3), with per-batch cache lengths and the
+  causal mask aligned to the newest positions.
 """
 from __future__ import annotations
 
@@ -69,6 +72,10 @@ def _load():
         lib.oracle_loss.argtypes = [_dp, _dp, _dp, _dp, ctypes.c_int, ctypes.c_int,
                                     ctypes.c_double, ctypes.c_int]
         lib.oracle_loss.restype = ctypes.c_double
+        lib.oracle_decode.argtypes = [_dp, _dp, _dp, _ip, ctypes.c_int, ctypes.c_int,
+                                      ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_double,
+                                      ctypes.c_int, _dp, _dp]
+        lib.oracle_decode.restype = None
         lib.oracle_num_threads.argtypes = []
         lib.oracle_num_threads.restype = ctypes.c_int
         lib.oracle_set_num_threads.argtypes = [ctypes.c_int]
@@ -157,6 +164,31 @@ def online_fwd(q_head, k_head, v_head, scale, causal=False, tile=128):
     lse = np.empty((N,), dtype=np.float64)
     _load().oracle_online_fwd(_p(q), _p(k), _p(v), N, d, float(scale), int(bool(causal)),
                               int(tile), _p(o), _p(lse))
+    return o, lse
+
+
+def decode(q, k_cache, v_cache, scale=None, causal=False, lens=None):
+    """Decode-shaped attention in fp64: q [B,H,Nq,d] against a cache
+    k_cache, v_cache [B,H,L,d] whose first lens[b] rows are valid (all L when
+    lens is None).  Causal: query i sees keys j <= lens[b] - Nq + i.  Returns
+    O [B,H,Nq,d] and lse [B,H,Nq]; a query that sees no key gets O = 0 and
+    lse = -inf."""
+    q, k, v = _f64(q), _f64(k_cache), _f64(v_cache)
+    B, H, Nq, d = _shape4(q)
+    L = k.shape[2]
+    if k.shape != (B, H, L, d) or v.shape != k.shape:
+        raise ValueError("k_cache and v_cache must be [B, H, L, d] with q's B, H, d")
+    lp = None
+    if lens is not None:
+        lens = np.ascontiguousarray(lens, dtype=np.int32)
+        if lens.shape != (B,) or lens.min() < 0 or lens.max() > L:
+            raise ValueError("lens must be [B] with 0 <= lens[b] <= L")
+        lp = lens.ctypes.data_as(_ip)
+    scale = default_scale(d) if scale is None else float(scale)
+    o = np.empty((B, H, Nq, d), dtype=np.float64)
+    lse = np.empty((B, H, Nq), dtype=np.float64)
+    _load().oracle_decode(_p(q), _p(k), _p(v), lp, B, H, Nq, L, d, scale, int(bool(causal)),
+                          _p(o), _p(lse))
     return o, lse
 
 

@@ -35,6 +35,17 @@
  *     page (running m, l, o; alpha = e^{m - m'}; p = e^{s - m'};
  *     l' = alpha l + sum p; o' = alpha o + p V_tile; O = o / l), written
  *     separately so a test can pin the three-pass definition against it.
+ *   - oracle_decode: the same attention for decode-shaped calls.  The first
+ *     page's §9.2 splits inference into prefill (a whole prompt at once) and
+ *     decode (one or a few new tokens per step); §9.3 says the KV cache keeps
+ *     the keys and values of every earlier token so that decode reads them
+ *     instead of recomputing them.  No formula is given; readings:
+ *       * a head's cache has L rows, of which the first len_b are valid for
+ *         batch b (all L when no lengths are given);
+ *       * the Nq queries are the newest Nq positions, so under the causal
+ *         mask query i sees keys j <= len_b - Nq + i (the mask's diagonal
+ *         ends at the last valid key);
+ *       * a query that sees no key gets O = 0 and lse = -inf.
  *
  * Layout: every tensor is [B, H, N, d] row-major (d contiguous), fp64; lse and
  * D are [B, H, N].  All loops are plain; OpenMP only splits independent rows
@@ -287,6 +298,47 @@ void oracle_online_fwd(const double *q, const double *k, const double *v,
     }
     free(sv);
     free(acc);
+  }
+}
+
+/* Decode-shaped attention: q, o [B,H,Nq,d]; k, v [B,H,L,d]; lse [B,H,Nq];
+ * lens [B] valid cache rows per batch (NULL: all L).  Three passes per query
+ * row over its visible keys, as in fwd_head. */
+void oracle_decode(const double *q, const double *k, const double *v,
+                   const int *lens, int B, int H, int Nq, int L, int d,
+                   double scale, int causal, double *o, double *lse) {
+  const i64 rows = (i64)B * H * Nq;
+#pragma omp parallel
+  {
+    double *s = (double *)malloc(sizeof(double) * (size_t)(L > 0 ? L : 1));
+#pragma omp for schedule(dynamic, 4)
+    for (i64 r = 0; r < rows; ++r) {
+      const i64 i = r % Nq, bh = r / Nq, b = bh / H;
+      const i64 len = lens ? lens[b] : L;
+      i64 cnt = causal ? len - Nq + i + 1 : len;
+      if (cnt < 0) cnt = 0;
+      const double *qi = q + r * d;
+      const double *kh = k + bh * (i64)L * d, *vh = v + bh * (i64)L * d;
+      double *oi = o + r * d;
+      for (i64 c = 0; c < d; ++c) oi[c] = 0.0;
+      if (cnt == 0) {
+        lse[r] = -INFINITY;
+        continue;
+      }
+      for (i64 j = 0; j < cnt; ++j) {
+        double acc = 0.0;
+        for (i64 c = 0; c < d; ++c) acc += qi[c] * kh[j * d + c];
+        s[j] = scale * acc;
+      }
+      double m;
+      double l = row_max_sum(s, cnt, &m);
+      for (i64 j = 0; j < cnt; ++j) {
+        double p = exp(s[j] - m) / l;
+        for (i64 c = 0; c < d; ++c) oi[c] += p * vh[j * d + c];
+      }
+      lse[r] = m + log(l);
+    }
+    free(s);
   }
 }
 
