@@ -21,6 +21,10 @@ by it.  Rank 0 prints one JSON line.
 
 --impl reference times the fp64 CPU oracle (the reference arm) on a bounded
 sample of the same workload, on the host cores.
+
+--decode WORKLOAD times fa_decode instead (a decode step of Nq new queries per
+head against a resident KV cache, same page §9.2-9.3) and prints its own line:
+bytes of cache read per second, against the measured HBM copy bandwidth.
 """
 from __future__ import annotations
 
@@ -43,9 +47,11 @@ import torch  # noqa: E402
 from tiled_attention_20_b200 import inputs, perf, ranks  # noqa: E402
 
 WORKLOAD = inputs.GPT_CAUSAL
+DECODE_WORKLOADS = {w.name: w for w in (inputs.DECODE_B8, inputs.DECODE_B8_RAGGED,
+                                        inputs.DECODE_SPEC, inputs.DECODE_LONG)}
 METRIC = "attention fwd+bwd TFLOP/s (bf16, causal, N=4096 d=128) and % of dense BF16 peak"
 UNIT = "TFLOP/s"
-KERNEL_SOURCES = ["fwd_kernel.cuh", "bwd_kernel.cuh", "dq_kernel.cuh", "sm100.cuh", "fa_api.cu"]
+KERNEL_SOURCES = ["fwd_kernel.cuh", "bwd_kernel.cuh", "dq_kernel.cuh", "decode_kernel.cuh", "sm100.cuh", "fa_api.cu"]
 
 
 def parse_args():
@@ -62,6 +68,9 @@ def parse_args():
     ap.add_argument("--no-e2e", action="store_true", help="skip the host-buffer leg (profiler runs)")
     ap.add_argument("--deterministic", action="store_true",
                     help="time fa_bwd_deterministic (bit-reproducible dQ) instead of fa_bwd")
+    ap.add_argument("--decode", default=None, metavar="WORKLOAD",
+                    choices=sorted(DECODE_WORKLOADS),
+                    help="time fa_decode on one decode workload instead of fwd+bwd")
     return ap.parse_args()
 
 
@@ -374,6 +383,158 @@ def run_ours(args, rank, world, local_rank, dist):
         print(json.dumps(line), flush=True)
 
 
+# ---------------------------------------------------------------- decode leg
+DECODE_METRIC = "decode attention cache-read bandwidth (bf16, KV cache in HBM)"
+DECODE_UNIT = "GB/s"
+
+
+def decode_bytes(w, lens) -> float:
+    """Algorithmic bytes of one decode call: every valid K and V row once,
+    q read, O (bf16) and lse (fp32) written."""
+    rows = float(sum(int(n) for n in lens)) * w.H
+    return rows * w.d * 2 * 2 + w.B * w.H * w.Nq * (w.d * 2 * 2 + 4)
+
+
+def cpu_oracle_decode_rate(q, k, v, lens, w, seconds: float):
+    """The oracle's decode (fp64, as it stands) on whole heads until `seconds`
+    of wall time have passed; returns (GB/s of algorithmic bytes, heads, cores, s)."""
+    import oracle  # CPU-baseline leg: one of the oracle's permitted users
+    t0 = time.time()
+    heads, done_bytes = 0, 0.0
+    while heads < w.B * w.H:
+        b, h = divmod(heads, w.H)
+        sl = lambda t: t[b:b + 1, h:h + 1]
+        oracle.decode(sl(q), sl(k), sl(v), causal=w.causal, lens=lens[b:b + 1].numpy())
+        done_bytes += int(lens[b]) * w.d * 2 * 2 + w.Nq * (w.d * 2 * 2 + 4)
+        heads += 1
+        if time.time() - t0 >= seconds:
+            break
+    el = time.time() - t0
+    return done_bytes / el / 1e9, heads, oracle.num_threads(), el
+
+
+def run_decode(args, rank, world, local_rank, dist):
+    import tiled_attention_20_b200.fa as fa
+    from tiled_attention_20_b200 import build as fa_build
+    if rank == 0 or world == 1:
+        fa_build.build()
+    if world > 1:
+        dist.barrier()
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    w = DECODE_WORKLOADS[args.decode]
+    q_h, k_h, v_h, lens_h = inputs.decode_qkv(w.B, w.H, w.Nq, w.L, w.d,
+                                              seed=ranks.rank_seed(w.seed, rank), ragged=w.ragged)
+    q, k, v = (t.to(dev) for t in (q_h, k_h, v_h))
+    lens = lens_h.to(dev) if w.ragged else None
+    o = torch.empty((w.B, w.H, w.Nq, w.d), dtype=torch.bfloat16, device=dev)
+    lse = torch.empty((w.B, w.H, w.Nq), dtype=torch.float32, device=dev)
+    ws = torch.zeros(max(fa.decode_workspace_size(w.B, w.H, w.Nq, w.L, w.d), 16),
+                     dtype=torch.uint8, device=dev)
+    splits, chunk = fa.decode_plan(w.B * w.H, w.Nq, w.L, w.d,
+                                   sms=torch.cuda.get_device_properties(dev).multi_processor_count)
+
+    def step():
+        fa.decode(q, k, v, cache_lens=lens, causal=w.causal, out=o, lse=lse, workspace=ws)
+
+    step()
+    fa.check_device_errors(dev)
+    if not torch.isfinite(o).all():
+        raise RuntimeError("non-finite decode output")
+    for _ in range(max(0, args.warmup - 1)):
+        step()
+    stream = torch.cuda.current_stream(dev)
+    sampler = ClockSampler(dev.index if world == 1 else local_rank)
+    sampler.start()
+    time.sleep(0.4)
+    for _ in range(max(3, args.warmup)):
+        step()
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize(dev)
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    fa.trace_start()
+    e0.record(stream)
+    for _ in range(args.steps):
+        step()
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    traced = fa.trace_stop()
+    if world > 1:
+        dist.barrier()
+    clocks = sampler.stop()
+    fa.check_device_errors(dev)
+    ms = ranks.max_over_ranks(e0.elapsed_time(e1) / args.steps, dist, dev)
+    nbytes = decode_bytes(w, lens_h.tolist())
+    value = nbytes * world / (ms * 1e-3) / 1e9
+    n_l, t_l = traced["fa_decode_kernel"]
+    launch_ms = t_l / n_l
+    peaks, peaks_src = measured_peaks()
+    achieved = nbytes / (launch_ms * 1e-3) / 1e9
+    roof = {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+            "frac": achieved / peaks["hbm_gbs"], "traffic": profiled_traffic(
+                "fa_decode_kernel:" + w.name), "kernel": "fa_decode_kernel",
+            "peak_source": f"{peaks_src} hbm_gbs (copy)", "launch_ms": launch_ms,
+            "algorithmic_bytes": nbytes}
+    kernels = {name: {"launches": n, "avg_ms": t / n} for name, (n, t) in traced.items()}
+
+    e2e = None
+    if not args.no_e2e:
+        # The cache is resident state; a step's inputs are its new queries and
+        # its results the attention output and lse.
+        hq = q_h.pin_memory()
+        ho = torch.empty(o.shape, dtype=torch.bfloat16).pin_memory()
+        hlse = torch.empty(lse.shape, dtype=torch.float32).pin_memory()
+
+        def e2e_step():
+            q.copy_(hq, non_blocking=True)
+            step()
+            ho.copy_(o, non_blocking=True)
+            hlse.copy_(lse, non_blocking=True)
+
+        e2e_step()
+        torch.cuda.synchronize(dev)
+        if world > 1:
+            dist.barrier()
+        n_e2e = max(1, args.e2e_steps)
+        e0.record(stream)
+        for _ in range(n_e2e):
+            e2e_step()
+        e1.record(stream)
+        torch.cuda.synchronize(dev)
+        ms_e2e = ranks.max_over_ranks(e0.elapsed_time(e1) / n_e2e, dist, dev)
+        nb = lambda *ts: sum(t.numel() * t.element_size() for t in ts)
+        e2e = {"value": nbytes * world / (ms_e2e * 1e-3) / 1e9, "unit": DECODE_UNIT,
+               "h2d_bytes_per_step": nb(hq), "d2h_bytes_per_step": nb(ho, hlse),
+               "steps": n_e2e, "ms_per_step": ms_e2e,
+               "api": "tiled_attention_20_b200.fa.decode (C ABI), cache resident"}
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        rate, heads, cores, el = cpu_oracle_decode_rate(q_h, k_h, v_h, lens_h, w, args.cpu_seconds)
+        cpu = {"value": rate, "unit": DECODE_UNIT, "cores": cores, "kind": "oracle",
+               "sample": f"{heads} of {w.B * w.H} heads of the workload in fp64, {el:.1f} s wall"}
+
+    if rank == 0:
+        cfg = {"workload": w.name, "B": w.B, "H": w.H, "Nq": w.Nq, "L": w.L, "d": w.d,
+               "causal": w.causal, "ragged": w.ragged, "seed": w.seed, "splits": splits,
+               "chunk_keys": chunk, "l2": "inputs_exceed_l2 (no flush)" if nbytes > 126e6
+               else "inputs_fit_l2",
+               "parallelism": f"heads replicated per GPU x{world}"}
+        line = {
+            "metric": DECODE_METRIC, "value": value, "unit": DECODE_UNIT, "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "bf16", "data": "synthetic", "config": cfg,
+            "pct_of_peak": value / world / peaks["hbm_gbs"],
+            "roofline": roof, "cpu_baseline": cpu, "e2e": e2e,
+            "gpu_launches": sum(n for n, _ in traced.values()), "kernels": kernels,
+            "clocks": clocks,
+        }
+        print(json.dumps(line), flush=True)
+
+
 def main():
     args = parse_args()
     info = ranks.rank_info()
@@ -388,7 +549,10 @@ def main():
         torch.cuda.set_device(local_rank)
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300))
     try:
-        run_ours(args, rank, world, local_rank, dist)
+        if args.decode:
+            run_decode(args, rank, world, local_rank, dist)
+        else:
+            run_ours(args, rank, world, local_rank, dist)
     finally:
         if dist is not None:
             dist.destroy_process_group()

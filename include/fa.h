@@ -50,10 +50,11 @@ typedef struct CUstream_st *fa_stream_t; /* same type as cudaStream_t */
 typedef enum {
   FA_OK = 0,
   FA_ERR_NULL = -1,           /* a required pointer is NULL */
-  FA_ERR_SHAPE = -2,          /* B, H or N < 1, or a tensor too large */
+  FA_ERR_SHAPE = -2,          /* B, H or N < 1, a tensor too large, or a decode
+                                 shape out of range (Nq, Nk, ld_kv, B*H) */
   FA_ERR_UNSUPPORTED_D = -3,  /* d not in {64, 128} */
   FA_ERR_ALIGN = -4,          /* a pointer is not 16-byte aligned */
-  FA_ERR_WORKSPACE = -5,      /* workspace smaller than fa_bwd_workspace_size */
+  FA_ERR_WORKSPACE = -5,      /* workspace smaller than its *_workspace_size */
   FA_ERR_LAUNCH = -6,         /* the CUDA runtime rejected a launch or query */
   FA_ERR_TIMEOUT = -7,        /* a device-side wait gave up (reported later) */
   FA_ERR_DEVICE_ASSERT = -8,  /* a device-side consistency check failed */
@@ -142,13 +143,59 @@ int fa_launch_shape(int pass, int B, int H, int N, int d, int causal,
                     int *ctas, int *work_units);
 
 /*
+ * Decode: attention of Nq new queries per head against a key/value cache
+ * ("第17讲 Tensor Core、HBM、SRAM 与 FlashAttention", §9.2 prefill and decode,
+ * §9.3 what the KV cache holds; the attention is the §8.1 formula).  The
+ * cache of each head is read once, split into chunks of keys handled by
+ * separate CTAs; the chunks' partial softmax states (m, l, o) are merged
+ * with the online-softmax rescaling of §8.3 by the last CTA of each head.
+ *   q           : bf16 [B,H,Nq,d], device, read only; 1 <= Nq <= 8.
+ *   k_cache,
+ *   v_cache     : bf16 [B,H,ld_kv,d], device, read only; rows 0 .. len_b-1 of
+ *                 each head are the cached keys / values of batch b.
+ *   o           : bf16 [B,H,Nq,d], device, written.
+ *   lse         : fp32 [B,H,Nq], device, written (natural log; -inf for a
+ *                 query that sees no key, whose o row is then 0).
+ *   cache_lens  : int32 [B], device, read only: len_b, the valid rows of
+ *                 batch b (values are clamped to [0, Nk]); NULL means every
+ *                 batch has Nk valid rows.
+ *   Nk          : the longest valid length, 1 <= Nk <= ld_kv (sets the split).
+ *   causal      : the Nq queries are the newest positions: query i sees keys
+ *                 j <= len_b - Nq + i.  Without it every valid key is seen.
+ *   num_splits  : chunks per head; 0 lets the library choose (wave-quantized
+ *                 to the SM count); otherwise it is rounded to whole 64-key
+ *                 tiles and capped by the chunk-size limit.
+ *   workspace   : device scratch of fa_decode_workspace_size(...) bytes with
+ *                 the same B, H, Nq, Nk, d and num_splits, 16-byte aligned,
+ *                 owned by the caller (NULL allowed when that size is 0).  Its
+ *                 first B*H 32-bit words are per-head counters that must be
+ *                 zero before the first call (cudaMemset once); each call
+ *                 leaves them zero again.  After FA_ERR_TIMEOUT, zero them
+ *                 again.  Calls sharing a workspace must not overlap on the GPU.
+ * The result is deterministic: the merge order is fixed.  B*H <= 65535.
+ */
+size_t fa_decode_workspace_size(int B, int H, int Nq, int Nk, int d, int num_splits);
+int fa_decode(const void *q, const void *k_cache, const void *v_cache, void *o,
+              float *lse, const int *cache_lens, int B, int H, int Nq, int Nk,
+              int ld_kv, int d, float scale, int causal, int num_splits,
+              void *workspace, size_t workspace_bytes, fa_stream_t stream);
+
+/* The split fa_decode uses for B*H heads on a device with `sms` SMs that
+ * hold `ctas_per_sm` decode CTAs each: *splits chunks of *chunk_keys keys
+ * per head (host arithmetic only, no device access).  Among chunk sizes of
+ * whole 64-key tiles up to the kernel's limit it picks the one with the
+ * fewest waves x (tiles per chunk + 1), ties going to longer chunks. */
+int fa_decode_plan(int BH, int Nq, int Nk, int d, int num_splits, int sms,
+                   int ctas_per_sm, int *splits, int *chunk_keys);
+
+/*
  * Opt-in per-kernel timing with CUDA events (a tracing aid; off by default).
  * After fa_trace_start(), every kernel the library enqueues, on any stream of
  * any device, is bracketed by two CUDA events recorded on its launch stream,
  * until fa_trace_stop().  fa_trace_stop() waits for those events and fills,
  * for each kernel id k < n_kernels, launches[k] and total_ms[k] (summed event
  * durations).  Kernel ids: 0 forward, 1 backward preprocess, 2 backward main,
- * 3 dQ conversion, 4 dQ pass of the deterministic backward
+ * 3 dQ conversion, 4 dQ pass of the deterministic backward, 5 decode
  * (fa_trace_kernel_name gives the kernel's name).  The
  * library creates the events on first use and reuses them afterwards; event
  * records add a few microseconds per launch.  fa_trace_start() discards a

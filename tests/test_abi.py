@@ -85,3 +85,46 @@ def test_no_device_means_launch_error_not_crash(lib):
         pytest.skip("a GPU is present")
     code = lib.fa_fwd(P, P, P, P, P, 1, 1, 16, 64, 0.125, 0, None)
     assert code in (-6, -9)
+
+
+# fa_decode(q, k, v, o, lse, lens, B, H, Nq, Nk, ld_kv, d, scale, causal, num_splits,
+#           workspace, workspace_bytes, stream): shape and pointer checks come
+# before any device access.
+@pytest.mark.parametrize("args,code", [
+    ((0, P, P, P, P, None, 1, 1, 1, 64, 64, 64, 0.1, 0, 0, None, 0, None), -1),   # NULL q
+    ((P, P, P, P, P, None, 1, 1, 0, 64, 64, 64, 0.1, 0, 0, None, 0, None), -2),   # Nq = 0
+    ((P, P, P, P, P, None, 1, 1, 9, 64, 64, 64, 0.1, 0, 0, None, 0, None), -2),   # Nq = 9
+    ((P, P, P, P, P, None, 1, 1, 1, 0, 64, 64, 0.1, 0, 0, None, 0, None), -2),    # Nk = 0
+    ((P, P, P, P, P, None, 1, 1, 1, 65, 64, 64, 0.1, 0, 0, None, 0, None), -2),   # ld < Nk
+    ((P, P, P, P, P, None, 300, 300, 1, 64, 64, 64, 0.1, 0, 0, None, 0, None), -2),  # B*H
+    ((P, P, P, P, P, None, 1, 1, 1, 64, 64, 96, 0.1, 0, 0, None, 0, None), -3),   # d = 96
+    ((P, P + 8, P, P, P, None, 1, 1, 1, 64, 64, 64, 0.1, 0, 0, None, 0, None), -4),  # misaligned k
+    ((P, P, P, P, P, P + 2, 1, 1, 1, 64, 64, 64, 0.1, 0, 0, None, 0, None), -4),  # misaligned lens
+    ((P, P, P, P, P, None, 1, 1, 1, 64, 64, 64, -1.0, 0, 0, None, 0, None), -10),  # scale < 0
+    ((P, P, P, P, P, None, 1, 1, 1, 64, 64, 64, 0.1, 0, -1, None, 0, None), -10),  # splits < 0
+])
+def test_decode_validation(lib, args, code):
+    assert lib.fa_decode(*args) == code
+
+
+def test_decode_plan(lib):
+    """The split covers every key with whole 64-key tiles, respects the
+    chunk limit (16 KB of scores: 4096 / padded Nq keys), honours a forced
+    split count, and fills but does not overflow one wave when that is best."""
+    import tiled_attention_20_b200.fa as fa
+    for BH, Nq, Nk, d in [(256, 1, 8192, 128), (32, 1, 8192, 128), (8, 4, 32768, 128),
+                          (2048, 1, 1024, 64), (1, 8, 100, 128), (64, 1, 131072, 128),
+                          (1, 1, 1, 64)]:
+        sp, ck = fa.decode_plan(BH, Nq, Nk, d)
+        nqp = 1 if Nq <= 1 else 2 if Nq <= 2 else 4 if Nq <= 4 else 8
+        assert ck % 64 == 0 and 64 <= ck <= 4096 // nqp
+        assert (sp - 1) * ck < Nk <= sp * ck
+    # 32 heads of an 8192-key cache on 148 SMs x 2 CTAs: one full wave.
+    sp, ck = fa.decode_plan(32, 1, 8192, 128)
+    assert 148 * 2 * 0.9 <= 32 * sp <= 148 * 2
+    # Forced counts round to whole tiles; a count above the tile count clamps.
+    assert fa.decode_plan(4, 1, 3000, 128, num_splits=7) == (7, 448)
+    assert fa.decode_plan(4, 1, 100, 128, num_splits=50) == (2, 64)
+    assert fa.decode_plan(4, 8, 100000, 128, num_splits=1) == (196, 512)
+    with pytest.raises(fa.FAError):
+        fa.decode_plan(4, 9, 100, 128)

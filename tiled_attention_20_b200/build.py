@@ -15,7 +15,7 @@ HERE = os.path.dirname(os.path.abspath(__file__))
 CSRC = os.path.join(HERE, "csrc")
 LIB = os.path.join(HERE, "libfa.so")
 SOURCES = ["fa_api.cu"]
-DEPS = ["fa_api.cu", "fwd_kernel.cuh", "bwd_kernel.cuh", "dq_kernel.cuh", "sm100.cuh"]
+DEPS = ["fa_api.cu", "fwd_kernel.cuh", "bwd_kernel.cuh", "dq_kernel.cuh", "decode_kernel.cuh", "sm100.cuh"]
 HEADER = os.path.join(os.path.dirname(HERE), "include", "fa.h")
 
 NVCC_FLAGS = [

@@ -14,6 +14,7 @@
 
 #include "../../include/fa.h"
 #include "bwd_kernel.cuh"
+#include "decode_kernel.cuh"
 #include "dq_kernel.cuh"
 #include "fwd_kernel.cuh"
 
@@ -45,9 +46,10 @@ EncodeTiledFn g_encode = nullptr;
 // Opt-in per-kernel timing: while enabled, every launch is bracketed by a
 // pair of CUDA events on its stream.
 enum { kKernFwd = 0, kKernBwdPrep = 1, kKernBwd = 2, kKernBwdConvert = 3, kKernDq = 4,
-       kNumKernels = 5 };
+       kKernDecode = 5, kNumKernels = 6 };
 const char* const kKernelNames[kNumKernels] = {"fa_fwd_kernel", "fa_bwd_prep", "fa_bwd_kernel",
-                                               "fa_bwd_dq_convert", "fa_dq_kernel"};
+                                               "fa_bwd_dq_convert", "fa_dq_kernel",
+                                               "fa_decode_kernel"};
 struct TraceRec {
   int kernel;
   int device;
@@ -341,6 +343,115 @@ int noalloc_scratch(void** out) {
   *out = g_noalloc_addr[dev];
   return FA_OK;
 }
+// ---------------------------------------------------------------- decode
+constexpr int kDecMaxNq = 8;
+
+int decode_max_chunk_tiles(int nqp) { return (4096 / nqp) / fa::kDecTileKeys; }
+
+int decode_plan(int BH, int Nq, int Nk, int num_splits, int sms, int per_sm, int* splits,
+                int* chunk) {
+  const int tiles = (Nk + fa::kDecTileKeys - 1) / fa::kDecTileKeys;
+  const int max_ct = decode_max_chunk_tiles(fa::dec_nqp(Nq));
+  int ct;
+  if (num_splits > 0) {
+    ct = (tiles + num_splits - 1) / num_splits;
+    ct = ct < 1 ? 1 : (ct > max_ct ? max_ct : ct);
+  } else {
+    // Wave quantization: the cost of a chunk size is the number of waves of
+    // CTAs times the tiles each CTA streams (+1 for its fixed work).
+    const long long slots = static_cast<long long>(sms) * per_sm;
+    long long best = -1;
+    ct = 1;
+    const int top = tiles < max_ct ? tiles : max_ct;
+    for (int c = 1; c <= top; ++c) {
+      const long long sp = (tiles + c - 1) / c;
+      const long long waves = (sp * BH + slots - 1) / slots;
+      const long long cost = waves * (c + 1);
+      if (best < 0 || cost <= best) {
+        best = cost;
+        ct = c;
+      }
+    }
+  }
+  *splits = (tiles + ct - 1) / ct;
+  *chunk = ct * fa::kDecTileKeys;
+  return FA_OK;
+}
+
+int check_decode_shape(int B, int H, int Nq, int Nk, int ld_kv, int d) {
+  if (B < 1 || H < 1 || Nq < 1 || Nq > kDecMaxNq || Nk < 1 || ld_kv < Nk) return FA_ERR_SHAPE;
+  if (d != 64 && d != 128) return FA_ERR_UNSUPPORTED_D;
+  if (static_cast<long long>(B) * H > 65535) return FA_ERR_SHAPE;
+  return FA_OK;
+}
+
+size_t decode_ws_bytes(int BH, int Nq, int d, int splits) {
+  if (splits <= 1) return 0;
+  const size_t nqp = static_cast<size_t>(fa::dec_nqp(Nq));
+  const size_t slots = static_cast<size_t>(BH) * splits * nqp;
+  return fa::round256(static_cast<size_t>(BH) * 4) + fa::round256(slots * d * 4) +
+         fa::round256(slots * 2 * 4);
+}
+
+template <int D, int NQP>
+int decode_occupancy(int* per_sm) {
+  auto kern = fa::fa_decode_kernel<D, NQP>;
+  const int smem = fa::DecLayout<D, NQP>::kSmemBytes;
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
+    return FA_ERR_LAUNCH;
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(per_sm, kern, fa::kDecThreads, smem) !=
+          cudaSuccess ||
+      *per_sm < 1)
+    return FA_ERR_LAUNCH;
+  return FA_OK;
+}
+
+int decode_occupancy_any(int d, int Nq, int* per_sm) {
+  switch (fa::dec_nqp(Nq) * (d == 64 ? 1 : -1)) {
+    case 1: return decode_occupancy<64, 1>(per_sm);
+    case 2: return decode_occupancy<64, 2>(per_sm);
+    case 4: return decode_occupancy<64, 4>(per_sm);
+    case 8: return decode_occupancy<64, 8>(per_sm);
+    case -1: return decode_occupancy<128, 1>(per_sm);
+    case -2: return decode_occupancy<128, 2>(per_sm);
+    case -4: return decode_occupancy<128, 4>(per_sm);
+    default: return decode_occupancy<128, 8>(per_sm);
+  }
+}
+
+template <int D, int NQP>
+int launch_decode_t(const fa::DecodeParams& p, int BH, cudaStream_t stream) {
+  auto kern = fa::fa_decode_kernel<D, NQP>;
+  const int smem = fa::DecLayout<D, NQP>::kSmemBytes;
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
+    return FA_ERR_LAUNCH;
+  LaunchTrace trace(kKernDecode, stream);
+  kern<<<dim3(p.splits, BH), fa::kDecThreads, smem, stream>>>(p);
+  return cudaPeekAtLastError() == cudaSuccess ? FA_OK : FA_ERR_LAUNCH;
+}
+
+int launch_decode(const fa::DecodeParams& p, int BH, int d, cudaStream_t stream) {
+  switch (fa::dec_nqp(p.Nq) * (d == 64 ? 1 : -1)) {
+    case 1: return launch_decode_t<64, 1>(p, BH, stream);
+    case 2: return launch_decode_t<64, 2>(p, BH, stream);
+    case 4: return launch_decode_t<64, 4>(p, BH, stream);
+    case 8: return launch_decode_t<64, 8>(p, BH, stream);
+    case -1: return launch_decode_t<128, 1>(p, BH, stream);
+    case -2: return launch_decode_t<128, 2>(p, BH, stream);
+    case -4: return launch_decode_t<128, 4>(p, BH, stream);
+    default: return launch_decode_t<128, 8>(p, BH, stream);
+  }
+}
+
+// Split of a decode problem on the current device.
+int decode_device_plan(int B, int H, int Nq, int Nk, int d, int num_splits, DeviceInfo** info,
+                       int* splits, int* chunk) {
+  int s = device_info(info);
+  if (s != FA_OK) return s;
+  int per_sm = 1;
+  if ((s = decode_occupancy_any(d, Nq, &per_sm)) != FA_OK) return s;
+  return decode_plan(B * H, Nq, Nk, num_splits, (*info)->sms, per_sm, splits, chunk);
+}
 }  // namespace
 
 extern "C" {
@@ -352,7 +463,7 @@ const char* fa_strerror(int status) {
     case FA_ERR_SHAPE: return "invalid shape (B, H, N must be >= 1 and B*H*N*d < 2^31)";
     case FA_ERR_UNSUPPORTED_D: return "unsupported head dimension (d must be 64 or 128)";
     case FA_ERR_ALIGN: return "a pointer is not 16-byte aligned";
-    case FA_ERR_WORKSPACE: return "workspace smaller than fa_bwd_workspace_size()";
+    case FA_ERR_WORKSPACE: return "workspace smaller than the *_workspace_size() it needs";
     case FA_ERR_LAUNCH: return "the CUDA runtime rejected a launch or query";
     case FA_ERR_TIMEOUT: return "a device-side wait timed out";
     case FA_ERR_DEVICE_ASSERT: return "a device-side consistency check failed";
@@ -362,6 +473,76 @@ const char* fa_strerror(int status) {
       return "problem needs more backward scratch than fa_bwd_noalloc's fixed maximum";
     default: return "unknown status";
   }
+}
+
+int fa_decode_plan(int BH, int Nq, int Nk, int d, int num_splits, int sms, int ctas_per_sm,
+                   int* splits, int* chunk_keys) {
+  if (!splits || !chunk_keys) return FA_ERR_NULL;
+  if (BH < 1 || BH > 65535 || Nq < 1 || Nq > kDecMaxNq || Nk < 1 || sms < 1 || ctas_per_sm < 1)
+    return FA_ERR_SHAPE;
+  if (d != 64 && d != 128) return FA_ERR_UNSUPPORTED_D;
+  return decode_plan(BH, Nq, Nk, num_splits, sms, ctas_per_sm, splits, chunk_keys);
+}
+
+size_t fa_decode_workspace_size(int B, int H, int Nq, int Nk, int d, int num_splits) {
+  if (check_decode_shape(B, H, Nq, Nk, Nk, d) != FA_OK) return 0;
+  DeviceInfo* info = nullptr;
+  int splits = 1, chunk = 0;
+  if (decode_device_plan(B, H, Nq, Nk, d, num_splits, &info, &splits, &chunk) != FA_OK) return 0;
+  return decode_ws_bytes(B * H, Nq, d, splits);
+}
+
+int fa_decode(const void* q, const void* k_cache, const void* v_cache, void* o, float* lse,
+              const int* cache_lens, int B, int H, int Nq, int Nk, int ld_kv, int d, float scale,
+              int causal, int num_splits, void* workspace, size_t workspace_bytes,
+              fa_stream_t stream) {
+  if (!q || !k_cache || !v_cache || !o || !lse) return FA_ERR_NULL;
+  int s = check_decode_shape(B, H, Nq, Nk, ld_kv, d);
+  if (s != FA_OK) return s;
+  if ((s = check_scale(scale)) != FA_OK) return s;
+  if (num_splits < 0) return FA_ERR_ARG;
+  if (!aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache) || !aligned16(o) ||
+      !aligned16(lse) || (cache_lens && (reinterpret_cast<uintptr_t>(cache_lens) & 3u)))
+    return FA_ERR_ALIGN;
+  DeviceInfo* info = nullptr;
+  int splits = 1, chunk = 0;
+  if ((s = decode_device_plan(B, H, Nq, Nk, d, num_splits, &info, &splits, &chunk)) != FA_OK)
+    return s;
+  const int BH = B * H;
+  const size_t need = decode_ws_bytes(BH, Nq, d, splits);
+  if (need > 0) {
+    if (!workspace) return FA_ERR_NULL;
+    if (!aligned16(workspace)) return FA_ERR_ALIGN;
+    if (workspace_bytes < need) return FA_ERR_WORKSPACE;
+  }
+  fa::DecodeParams p;
+  p.q = static_cast<const uint16_t*>(q);
+  p.k = static_cast<const uint16_t*>(k_cache);
+  p.v = static_cast<const uint16_t*>(v_cache);
+  p.o = static_cast<uint16_t*>(o);
+  p.lse = lse;
+  p.lens = cache_lens;
+  p.counter = nullptr;
+  p.part_o = p.part_ml = nullptr;
+  if (need > 0) {
+    const size_t nqp = static_cast<size_t>(fa::dec_nqp(Nq));
+    const size_t slots = static_cast<size_t>(BH) * splits * nqp;
+    uint8_t* ws = static_cast<uint8_t*>(workspace);
+    p.counter = reinterpret_cast<int*>(ws);
+    p.part_o = reinterpret_cast<float*>(ws + fa::round256(static_cast<size_t>(BH) * 4));
+    p.part_ml = reinterpret_cast<float*>(ws + fa::round256(static_cast<size_t>(BH) * 4) +
+                                         fa::round256(slots * d * 4));
+  }
+  p.status = info->status;
+  p.H = H;
+  p.Nq = Nq;
+  p.Nk = Nk;
+  p.ld = ld_kv;
+  p.splits = splits;
+  p.chunk = chunk;
+  p.scale_log2 = scale * 1.4426950408889634f;
+  p.causal = causal ? 1 : 0;
+  return launch_decode(p, BH, d, reinterpret_cast<cudaStream_t>(stream));
 }
 
 int fa_launch_shape(int pass, int B, int H, int N, int d, int causal, int* ctas, int* work_units) {

@@ -27,10 +27,12 @@ STATUS_NAMES = {
 
 EXPORTED = ["fa_fwd", "fa_bwd", "fa_bwd_workspace_size", "fa_strerror",
             "fa_check_device_errors", "fa_launch_shape", "fa_trace_start", "fa_trace_stop",
-            "fa_trace_kernel_name", "fa_bwd_noalloc", "fa_bwd_deterministic"]
+            "fa_trace_kernel_name", "fa_bwd_noalloc", "fa_bwd_deterministic",
+            "fa_decode", "fa_decode_workspace_size", "fa_decode_plan"]
 NOALLOC_MAX_SCRATCH = 32 << 20  # FA_BWD_NOALLOC_MAX_SCRATCH
 KERNEL_IDS = {0: "fa_fwd_kernel", 1: "fa_bwd_prep", 2: "fa_bwd_kernel", 3: "fa_bwd_dq_convert",
-              4: "fa_dq_kernel"}
+              4: "fa_dq_kernel", 5: "fa_decode_kernel"}
+DECODE_MAX_NQ = 8
 
 
 class FAError(RuntimeError):
@@ -77,6 +79,14 @@ def load(path: str = LIB_PATH):
         lib.fa_bwd_noalloc.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp,
                                        _i, _i, _i, _i, _f, _i, _i, _vp]
         lib.fa_bwd_noalloc.restype = _i
+        lib.fa_decode.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _f, _i,
+                                  _i, _vp, _sz, _vp]
+        lib.fa_decode.restype = _i
+        lib.fa_decode_workspace_size.argtypes = [_i, _i, _i, _i, _i, _i]
+        lib.fa_decode_workspace_size.restype = _sz
+        lib.fa_decode_plan.argtypes = [_i, _i, _i, _i, _i, _i, _i, ctypes.POINTER(_i),
+                                       ctypes.POINTER(_i)]
+        lib.fa_decode_plan.restype = _i
         _lib = lib
     return _lib
 
@@ -214,3 +224,57 @@ def trace_stop() -> dict:
     _check(load().fa_trace_stop(n, launches, ms), "fa_trace_stop")
     return {load().fa_trace_kernel_name(k).decode(): (launches[k], ms[k])
             for k in range(n) if launches[k]}
+
+
+def decode_plan(BH, Nq, Nk, d, num_splits=0, sms=148, ctas_per_sm=2):
+    """(splits, chunk_keys) fa_decode picks for this shape on a device with
+    ``sms`` SMs holding ``ctas_per_sm`` decode CTAs each (host arithmetic)."""
+    sp, ck = _i(0), _i(0)
+    _check(load().fa_decode_plan(BH, Nq, Nk, d, num_splits, sms, ctas_per_sm,
+                                 ctypes.byref(sp), ctypes.byref(ck)), "fa_decode_plan")
+    return sp.value, ck.value
+
+
+def decode_workspace_size(B, H, Nq, Nk, d, num_splits=0) -> int:
+    """Bytes of scratch fa_decode needs on the current device (0: none)."""
+    return int(load().fa_decode_workspace_size(B, H, Nq, Nk, d, num_splits))
+
+
+def decode(q, k_cache, v_cache, cache_lens=None, scale=None, causal=False, nk=None,
+           num_splits=0, out=None, lse=None, workspace=None):
+    """Decode-shaped attention (fa_decode): q [B,H,Nq,d] (Nq <= 8) against a
+    cache k_cache, v_cache [B,H,ld,d].  nk (default ld) is the longest valid
+    length; cache_lens (int32 [B] on the device, optional) the valid rows per
+    batch.  Returns O [B,H,Nq,d] bf16 and lse [B,H,Nq] fp32.  ``workspace``
+    (uint8, at least decode_workspace_size bytes, its first B*H int32 words
+    zero) may be kept across calls; without one a zeroed buffer is made."""
+    for t in (q, k_cache, v_cache):
+        if not t.is_cuda or t.dtype != torch.bfloat16 or not t.is_contiguous() or t.dim() != 4:
+            raise ValueError("q, k_cache, v_cache must be contiguous bf16 [B, H, *, d] CUDA tensors")
+        if t.device != q.device:
+            raise ValueError("inputs must be on one device")
+    B, H, Nq, d = q.shape
+    ld = k_cache.shape[2]
+    if k_cache.shape != (B, H, ld, d) or v_cache.shape != k_cache.shape:
+        raise ValueError("k_cache and v_cache must be [B, H, ld, d] with q's B, H, d")
+    nk = ld if nk is None else int(nk)
+    if cache_lens is not None:
+        if (not cache_lens.is_cuda or cache_lens.dtype != torch.int32 or cache_lens.numel() != B
+                or not cache_lens.is_contiguous()):
+            raise ValueError("cache_lens must be a contiguous int32 [B] CUDA tensor")
+    scale = default_scale(d) if scale is None else float(scale)
+    if out is None:
+        out = torch.empty((B, H, Nq, d), dtype=torch.bfloat16, device=q.device)
+    if lse is None:
+        lse = torch.empty((B, H, Nq), dtype=torch.float32, device=q.device)
+    with torch.cuda.device(q.device):
+        if workspace is None:
+            ws_bytes = decode_workspace_size(B, H, Nq, nk, d, num_splits)
+            workspace = torch.zeros(max(ws_bytes, 16), dtype=torch.uint8, device=q.device)
+        st = load().fa_decode(q.data_ptr(), k_cache.data_ptr(), v_cache.data_ptr(),
+                              out.data_ptr(), lse.data_ptr(),
+                              None if cache_lens is None else cache_lens.data_ptr(),
+                              B, H, Nq, nk, ld, d, scale, int(bool(causal)), int(num_splits),
+                              workspace.data_ptr(), workspace.numel(), _stream(q.device))
+    _check(st, "fa_decode")
+    return out, lse

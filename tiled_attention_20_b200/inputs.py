@@ -14,6 +14,11 @@ Recipe (one generator per call, seeded with ``seed``):
    ``torch.randperm`` from the same generator, are multiplied by 8.  V and dO
    keep standard deviation 1.
 3. Everything is rounded to bf16 (round to nearest even).
+
+Decode inputs (``decode_qkv``): one generator per call; ``torch.randn`` fp32
+for q [B, H, Nq, d], then the caches k, v [B, H, L, d]; with ``ragged`` the
+per-batch valid lengths are then drawn uniformly from [L/2, L] with
+``torch.randint`` (else every batch has L rows); bf16 rounding last.
 """
 from __future__ import annotations
 
@@ -44,6 +49,44 @@ MID_C = Workload("fwdbwd_c_B4_H16_N1024_d64", 4, 16, 1024, 64, True, True)
 GPT_CAUSAL = Workload("fwdbwd_c_B2_H32_N4096_d128", 2, 32, 4096, 128, True, True)
 LONG_CONTEXT = Workload("fwdbwd_c_B1_H16_N16384_d128_lc", 1, 16, 16384, 128, True, True,
                         dist="long_context")
+
+
+@dataclass(frozen=True)
+class DecodeWorkload:
+    """A decode step: Nq new queries per head against an L-row cache."""
+    name: str
+    B: int
+    H: int
+    Nq: int
+    L: int
+    d: int
+    causal: bool
+    ragged: bool = False
+    seed: int = 0
+
+
+# Decode-shaped calls: GPT-style heads (H=32, d=128) at batch 8 reading an
+# 8192-token cache (1 GiB of K and V, well above L2), its ragged-length and
+# speculative (Nq=4, causal) variants, and a small-batch long-cache case.
+DECODE_B8 = DecodeWorkload("decode_B8_H32_Nq1_L8192_d128", 8, 32, 1, 8192, 128, False)
+DECODE_B8_RAGGED = DecodeWorkload("decode_B8_H32_Nq1_L8192_d128_ragged", 8, 32, 1, 8192, 128,
+                                  False, ragged=True)
+DECODE_SPEC = DecodeWorkload("decode_B8_H32_Nq4_L8192_d128_causal", 8, 32, 4, 8192, 128, True)
+DECODE_LONG = DecodeWorkload("decode_B1_H32_Nq1_L65536_d128", 1, 32, 1, 65536, 128, False)
+
+
+def decode_qkv(B: int, H: int, Nq: int, L: int, d: int, seed: int = 0, ragged: bool = False):
+    """(q, k_cache, v_cache, lens): bf16 [B,H,Nq,d], [B,H,L,d], [B,H,L,d] and
+    int32 [B] valid lengths."""
+    g = torch.Generator(device="cpu").manual_seed(int(seed))
+    q = torch.randn((B, H, Nq, d), generator=g, dtype=torch.float32)
+    k = torch.randn((B, H, L, d), generator=g, dtype=torch.float32)
+    v = torch.randn((B, H, L, d), generator=g, dtype=torch.float32)
+    if ragged:
+        lens = torch.randint(L // 2, L + 1, (B,), generator=g, dtype=torch.int32)
+    else:
+        lens = torch.full((B,), L, dtype=torch.int32)
+    return q.to(torch.bfloat16), k.to(torch.bfloat16), v.to(torch.bfloat16), lens
 
 
 def sweep_workloads():
