@@ -15,6 +15,7 @@ are stated in the C file's header:
 * lse = m + ln l per row (natural log of the scaled scores);
 * backward: the exact gradient of sum(O * dO) (pages silent; calculus);
 * ``online_fwd``: the online-softmax recurrence of the same page's §8.3;
+* ``gemm``: the plain matrix product (the CS336 lecture's opening curve);
 * ``decode``: the same attention for a few new queries against a key/value
   cache (the same page's §9.2–9.3), with per-batch cache lengths and the
   causal mask aligned to the newest positions.
@@ -76,6 +77,8 @@ def _load():
                                       ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_double,
                                       ctypes.c_int, _dp, _dp]
         lib.oracle_decode.restype = None
+        lib.oracle_gemm.argtypes = [_dp, _dp, _dp, ctypes.c_int, ctypes.c_int, ctypes.c_int]
+        lib.oracle_gemm.restype = None
         lib.oracle_num_threads.argtypes = []
         lib.oracle_num_threads.restype = ctypes.c_int
         lib.oracle_set_num_threads.argtypes = [ctypes.c_int]
@@ -190,6 +193,18 @@ def decode(q, k_cache, v_cache, scale=None, causal=False, lens=None):
     _load().oracle_decode(_p(q), _p(k), _p(v), lp, B, H, Nq, L, d, scale, int(bool(causal)),
                           _p(o), _p(lse))
     return o, lse
+
+
+def gemm(a, b):
+    """C = A B in fp64 for A [M, K] and B [K, N] (plain triple loop)."""
+    a, b = _f64(a), _f64(b)
+    if a.ndim != 2 or b.ndim != 2 or a.shape[1] != b.shape[0]:
+        raise ValueError("expected A [M, K] and B [K, N]")
+    M, K = a.shape
+    N = b.shape[1]
+    c = np.empty((M, N), dtype=np.float64)
+    _load().oracle_gemm(_p(a), _p(b), _p(c), M, N, K)
+    return c
 
 
 def loss(q_head, k_head, v_head, dO_head, scale, causal=False) -> float:

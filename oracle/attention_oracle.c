@@ -35,6 +35,8 @@
  *     page (running m, l, o; alpha = e^{m - m'}; p = e^{s - m'};
  *     l' = alpha l + sum p; o' = alpha o + p V_tile; O = o / l), written
  *     separately so a test can pin the three-pass definition against it.
+ *   - oracle_gemm: the plain matrix product C = A B (the matrix multiply
+ *     whose throughput curve the CS336 lecture opens with).
  *   - oracle_decode: the same attention for decode-shaped calls.  The first
  *     page's §9.2 splits inference into prefill (a whole prompt at once) and
  *     decode (one or a few new tokens per step); §9.3 says the KV cache keeps
@@ -339,6 +341,25 @@ void oracle_decode(const double *q, const double *k, const double *v,
       lse[r] = m + log(l);
     }
     free(s);
+  }
+}
+
+/* Plain matrix product C = A B in fp64: A [M,K], B [K,N], C [M,N], all
+ * row-major.  The operation whose throughput-versus-size curve opens
+ * "CS336 Lecture 5 · GPUs, TPUs" (notes, opening goal and "矩阵谜题"); its
+ * cost, 2MKN, is "第17讲 Tensor Core、HBM、SRAM 与 FlashAttention" §5.3.
+ * C_ij = sum_k A_ik B_kj, summed in k order. */
+void oracle_gemm(const double *A, const double *B, double *C, int M, int N,
+                 int K) {
+#pragma omp parallel for schedule(static)
+  for (i64 i = 0; i < M; ++i) {
+    double *ci = C + i * N;
+    for (i64 j = 0; j < N; ++j) ci[j] = 0.0;
+    for (i64 k = 0; k < K; ++k) {
+      const double a = A[i * K + k];
+      const double *bk = B + k * N;
+      for (i64 j = 0; j < N; ++j) ci[j] += a * bk[j];
+    }
   }
 }
 
