@@ -22,6 +22,13 @@ by it.  Rank 0 prints one JSON line.
 --impl reference times the fp64 CPU oracle (the reference arm) on a bounded
 sample of the same workload, on the host cores.
 
+--fp8 times fa_fwd_fp8 (E4M3 Q, K, V, per-head descale factors) on the same
+shape, forward only, against twice the measured bf16 peak.
+
+--gemm-sweep times fa_gemm on square sizes N = 256 i + {0, 1, 2, 8, 16}
+(the lecture's divisibility classes) up to 8192 and prints the curve in the
+same JSON line, with cuBLAS beside it; value = TFLOP/s at N = 8192.
+
 --decode WORKLOAD times fa_decode instead (a decode step of Nq new queries per
 head against a resident KV cache, same page §9.2-9.3) and prints its own line:
 bytes of cache read per second, against the measured HBM copy bandwidth.
@@ -71,6 +78,10 @@ def parse_args():
     ap.add_argument("--no-e2e", action="store_true", help="skip the host-buffer leg (profiler runs)")
     ap.add_argument("--deterministic", action="store_true",
                     help="time fa_bwd_deterministic (bit-reproducible dQ) instead of fa_bwd")
+    ap.add_argument("--gemm-sweep", action="store_true",
+                    help="time fa_gemm on square sizes of every divisibility class instead")
+    ap.add_argument("--fp8", action="store_true",
+                    help="time fa_fwd_fp8 (E4M3 operands) on the benchmark shape instead")
     ap.add_argument("--decode", default=None, metavar="WORKLOAD",
                     choices=sorted(DECODE_WORKLOADS),
                     help="time fa_decode on one decode workload instead of fwd+bwd")
@@ -416,6 +427,271 @@ def cpu_oracle_decode_rate(q, k, v, lens, w, seconds: float):
     return done_bytes / el / 1e9, heads, oracle.num_threads(), el
 
 
+# ---------------------------------------------------------------- GEMM sweep
+GEMM_METRIC = "bf16 GEMM TFLOP/s, square N x N x N (256x128 tiles, persistent over the SMs)"
+
+
+def gemm_div_class(n: int) -> int:
+    """Largest of 32, 16, 8, 2, 1 that divides n (the lecture's colour classes)."""
+    for c in (32, 16, 8, 2):
+        if n % c == 0:
+            return c
+    return 1
+
+
+def run_gemm_sweep(args, rank, world, local_rank, dist):
+    """Throughput of fa_gemm against the square size N, for N = 256 i + delta
+    (i = 1..32, delta in 0, 1, 2, 8, 16: divisibility classes 32+, 1, 2, 8,
+    16), each point the mean of `reps` launches with L2 flushed before each;
+    torch.matmul (cuBLAS) is timed beside it for context."""
+    import tiled_attention_20_b200.fa as fa
+    from tiled_attention_20_b200 import build as fa_build
+    if rank == 0 or world == 1:
+        fa_build.build()
+    if world > 1:
+        dist.barrier()
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    sms = torch.cuda.get_device_properties(dev).multi_processor_count
+    stream = torch.cuda.current_stream(dev)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)  # > 126 MB of L2
+    g = torch.Generator(device=dev).manual_seed(ranks.rank_seed(0, rank))
+    peaks, peaks_src = measured_peaks()
+    reps = max(3, min(args.steps, 10))
+    ws = torch.empty(320 << 20, dtype=torch.uint8, device=dev)  # aligned copies up to N = 8208
+    n_warm = max(2, min(args.warmup, 3))
+
+    def timed(fn):
+        for _ in range(n_warm):
+            fn()
+        tot = 0.0
+        for _ in range(reps):
+            flush.zero_()
+            e0 = torch.cuda.Event(enable_timing=True)
+            e1 = torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            fn()
+            e1.record(stream)
+            e1.synchronize()
+            tot += e0.elapsed_time(e1)
+        return tot / reps
+
+    sampler = ClockSampler(dev.index if world == 1 else local_rank)
+    sampler.start()
+    time.sleep(0.4)
+    sweep = []
+    sizes = [256 * i + dlt for i in range(1, 33) for dlt in (0, 1, 2, 8, 16)]
+    launches = 0
+    for n in sizes:
+        a = torch.randn((n, n), generator=g, device=dev, dtype=torch.float32).to(torch.bfloat16)
+        b = torch.randn((n, n), generator=g, device=dev, dtype=torch.float32).to(torch.bfloat16)
+        c = torch.empty((n, n), dtype=torch.bfloat16, device=dev)
+        ms = timed(lambda: fa.gemm(a, b, out=c, workspace=ws))
+        ms_cublas = timed(lambda: torch.matmul(a, b, out=c))
+        tm, tn = fa.gemm_tiles(n, n)
+        launches += (n_warm + reps) * (1 if n % 8 == 0 else 3)  # GEMM (+ two aligned copies)
+        fl = 2.0 * n * n * n
+        sweep.append({"N": n, "div": gemm_div_class(n), "tiles": tm * tn,
+                      "rounds": -(-(tm * tn) // sms), "ms": ms, "tflops": fl / ms / 1e9,
+                      "cublas_tflops": fl / ms_cublas / 1e9})
+    clocks = sampler.stop()
+    fa.check_device_errors(dev)
+    top = next(r for r in sweep if r["N"] == 8192)
+    value = top["tflops"] * world
+    roof = {"bound": "tensor", "achieved": top["tflops"], "peak": peaks["bf16_tflops"],
+            "unit": "TFLOP/s", "frac": top["tflops"] / peaks["bf16_tflops"], "traffic": None,
+            "kernel": "fa_gemm_kernel", "peak_source": f"{peaks_src} bf16_tflops (burst)",
+            "launch_ms": top["ms"], "at": "N=8192"}
+
+    e2e = None
+    if not args.no_e2e:
+        n = 8192
+        ha = torch.randn((n, n), generator=torch.Generator().manual_seed(1)).to(torch.bfloat16).pin_memory()
+        hb = torch.randn((n, n), generator=torch.Generator().manual_seed(2)).to(torch.bfloat16).pin_memory()
+        hc = torch.empty((n, n), dtype=torch.bfloat16).pin_memory()
+        a = torch.empty_like(ha, device=dev)
+        b = torch.empty_like(hb, device=dev)
+        c = torch.empty((n, n), dtype=torch.bfloat16, device=dev)
+
+        def e2e_step():
+            a.copy_(ha, non_blocking=True)
+            b.copy_(hb, non_blocking=True)
+            fa.gemm(a, b, out=c, workspace=ws)
+            hc.copy_(c, non_blocking=True)
+
+        e2e_step()
+        torch.cuda.synchronize(dev)
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        k = max(1, args.e2e_steps)
+        e0.record(stream)
+        for _ in range(k):
+            e2e_step()
+        e1.record(stream)
+        torch.cuda.synchronize(dev)
+        ms_e2e = e0.elapsed_time(e1) / k
+        e2e = {"value": 2.0 * n ** 3 / ms_e2e / 1e9 * world, "unit": UNIT,
+               "h2d_bytes_per_step": 2 * n * n * 2, "d2h_bytes_per_step": n * n * 2,
+               "steps": k, "ms_per_step": ms_e2e, "api": "tiled_attention_20_b200.fa.gemm (C ABI)"}
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        import oracle  # CPU-baseline leg: the fp64 oracle's plain product
+        n = 1024
+        a = torch.randn((n, n), generator=torch.Generator().manual_seed(3)).to(torch.bfloat16)
+        t0 = time.time()
+        done = 0
+        while time.time() - t0 < args.cpu_seconds:
+            oracle.gemm(a, a)
+            done += 1
+        el = time.time() - t0
+        cpu = {"value": 2.0 * n ** 3 * done / el / 1e12, "unit": UNIT,
+               "cores": oracle.num_threads(), "kind": "oracle",
+               "sample": f"{done} products of {n} x {n} x {n} in fp64, {el:.1f} s wall"}
+
+    if rank == 0:
+        line = {
+            "metric": GEMM_METRIC, "value": value, "unit": UNIT, "n_gpus": world,
+            "steps": reps, "warmup": args.warmup, "ms_per_step": top["ms"],
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "bf16", "data": "synthetic",
+            "config": {"workload": "gemm_square_sweep_N256_to_8208", "value_at": "N=8192",
+                       "tile": "256x128", "sms": sms, "l2": "flushed before every timed launch",
+                       "parallelism": f"replicated per GPU x{world}"},
+            "pct_of_peak": top["tflops"] / peaks["bf16_tflops"],
+            "roofline": roof, "cpu_baseline": cpu, "e2e": e2e,
+            "gpu_launches": launches, "clocks": clocks, "sweep": sweep,
+        }
+        print(json.dumps(line), flush=True)
+
+
+# ---------------------------------------------------------------- FP8 leg
+FP8_METRIC = "attention fwd TFLOP/s (fp8 e4m3 operands, causal, N=4096 d=128)"
+
+
+def run_fp8(args, rank, world, local_rank, dist):
+    """fa_fwd_fp8 on the benchmark workload's shape: E4M3 Q, K, V with
+    per-head descale factors (inputs.fp8_qkv), bf16 O, fp32 lse."""
+    import tiled_attention_20_b200.fa as fa
+    from tiled_attention_20_b200 import build as fa_build
+    if rank == 0 or world == 1:
+        fa_build.build()
+    if world > 1:
+        dist.barrier()
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    w = WORKLOAD
+    host = inputs.fp8_qkv(w.B, w.H, w.N, w.d, seed=ranks.rank_seed(w.seed, rank), dist=w.dist)
+    q8, k8, v8, fq, fk, fv = (t.to(dev) for t in host)
+    o = torch.empty((w.B, w.H, w.N, w.d), dtype=torch.bfloat16, device=dev)
+    lse = torch.empty((w.B, w.H, w.N), dtype=torch.float32, device=dev)
+
+    def step():
+        fa.fwd_fp8(q8, k8, v8, fq, fk, fv, causal=w.causal, out=o, lse=lse)
+
+    step()
+    fa.check_device_errors(dev)
+    if not torch.isfinite(o).all():
+        raise RuntimeError("non-finite FP8 output")
+    for _ in range(max(0, args.warmup - 1)):
+        step()
+    stream = torch.cuda.current_stream(dev)
+    sampler = ClockSampler(dev.index if world == 1 else local_rank)
+    sampler.start()
+    time.sleep(0.4)
+    for _ in range(max(3, args.warmup)):
+        step()
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize(dev)
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    fa.trace_start()
+    e0.record(stream)
+    for _ in range(args.steps):
+        step()
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    traced = fa.trace_stop()
+    if world > 1:
+        dist.barrier()
+    clocks = sampler.stop()
+    fa.check_device_errors(dev)
+    ms = ranks.max_over_ranks(e0.elapsed_time(e1) / args.steps, dist, dev)
+    flops = perf.attention_flops(w.B, w.H, w.N, w.d, w.causal, False)
+    value = ranks.weak_scaling_rate(flops, world, ms) / 1e12
+    n_l, t_l = traced["fa_fwd_kernel"]
+    launch_ms = t_l / n_l
+    peaks, peaks_src = measured_peaks()
+    peak8 = 2.0 * peaks["bf16_tflops"]  # nominal dense fp8 / bf16 ratio: 4.5 / 2.25
+    achieved = flops / (launch_ms * 1e-3) / 1e12
+    roof = {"bound": "tensor", "achieved": achieved, "peak": peak8, "unit": "TFLOP/s",
+            "frac": achieved / peak8, "traffic": None, "kernel": "fa_fwd_kernel (fp8)",
+            "peak_source": f"{peaks_src} bf16_tflops (burst) x 2, the nominal fp8/bf16 ratio",
+            "launch_ms": launch_ms}
+    kernels = {name: {"launches": n, "avg_ms": t / n} for name, (n, t) in traced.items()}
+
+    e2e = None
+    if not args.no_e2e:
+        hin = [t.pin_memory() for t in host[:3]]
+        ho = torch.empty(o.shape, dtype=torch.bfloat16).pin_memory()
+        hlse = torch.empty(lse.shape, dtype=torch.float32).pin_memory()
+
+        def e2e_step():
+            for dst, src in zip((q8, k8, v8), hin):
+                dst.copy_(src, non_blocking=True)
+            step()
+            ho.copy_(o, non_blocking=True)
+            hlse.copy_(lse, non_blocking=True)
+
+        e2e_step()
+        torch.cuda.synchronize(dev)
+        n_e2e = max(1, args.e2e_steps)
+        e0.record(stream)
+        for _ in range(n_e2e):
+            e2e_step()
+        e1.record(stream)
+        torch.cuda.synchronize(dev)
+        ms_e2e = ranks.max_over_ranks(e0.elapsed_time(e1) / n_e2e, dist, dev)
+        nb = lambda *ts: sum(t.numel() * t.element_size() for t in ts)
+        e2e = {"value": ranks.weak_scaling_rate(flops, world, ms_e2e) / 1e12, "unit": UNIT,
+               "h2d_bytes_per_step": nb(*hin), "d2h_bytes_per_step": nb(ho, hlse),
+               "steps": n_e2e, "ms_per_step": ms_e2e,
+               "api": "tiled_attention_20_b200.fa.fwd_fp8 (C ABI)"}
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        import oracle  # CPU-baseline leg: the fp64 oracle on the dequantised inputs
+        t0 = time.time()
+        heads = 0
+        while heads < w.B * w.H and time.time() - t0 < args.cpu_seconds:
+            b, h = divmod(heads, w.H)
+            deq = [host[i][b:b + 1, h:h + 1].to(torch.float64) * float(host[3 + i][b, h])
+                   for i in range(3)]
+            oracle.fwd(*deq, causal=w.causal)
+            heads += 1
+        el = time.time() - t0
+        cpu = {"value": perf.attention_flops(1, 1, w.N, w.d, w.causal, False) * heads / el / 1e12,
+               "unit": UNIT, "cores": oracle.num_threads(), "kind": "oracle",
+               "sample": f"{heads} of {w.B * w.H} heads, forward in fp64 on the dequantised "
+                         f"inputs, {el:.1f} s wall"}
+
+    if rank == 0:
+        line = {
+            "metric": FP8_METRIC, "value": value, "unit": UNIT, "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "e4m3", "data": "synthetic",
+            "config": workload_config(w, {"passes": "fwd", "operands": "e4m3, per-head descale",
+                                          "parallelism": f"heads replicated per GPU x{world}"}),
+            "pct_of_peak": value / world / peak8,
+            "roofline": roof, "cpu_baseline": cpu, "e2e": e2e,
+            "gpu_launches": sum(n for n, _ in traced.values()), "kernels": kernels,
+            "clocks": clocks,
+        }
+        print(json.dumps(line), flush=True)
+
+
 def run_decode(args, rank, world, local_rank, dist):
     import tiled_attention_20_b200.fa as fa
     from tiled_attention_20_b200 import build as fa_build
@@ -554,6 +830,10 @@ def main():
     try:
         if args.decode:
             run_decode(args, rank, world, local_rank, dist)
+        elif args.fp8:
+            run_fp8(args, rank, world, local_rank, dist)
+        elif args.gemm_sweep:
+            run_gemm_sweep(args, rank, world, local_rank, dist)
         else:
             run_ours(args, rank, world, local_rank, dist)
     finally:

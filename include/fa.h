@@ -77,6 +77,28 @@ int fa_fwd(const void *q, const void *k, const void *v, void *o, float *lse,
            fa_stream_t stream);
 
 /*
+ * Forward with FP8 operands: O = softmax(scale * Q K^T [+ causal]) V where
+ * Q, K and V are given as E4M3 values with one fp32 dequantisation factor per
+ * (b, h) each (the real value is e4m3 * descale).  The low-precision trick
+ * of "第17讲 Tensor Core、HBM、SRAM 与 FlashAttention" §4.4 (FP8 on the tensor
+ * cores, twice the BF16 rate) applied to both GEMMs: S = Q K^T from E4M3
+ * operands with fp32 accumulation, and O += P V with P rounded to E4M3.  O
+ * is normalised by the sum of the rounded P, so each output row is a convex
+ * combination of V rows; lse uses the unrounded P.  Accuracy is set by the
+ * E4M3 rounding of P (relative 2^-4); see the library's design notes.
+ *   q, k, v     : E4M3 [B,H,N,d], device, read only; d must be 128.
+ *   descale_q,
+ *   descale_k,
+ *   descale_v   : fp32 [B*H], device, read only (4-byte aligned).
+ *   o           : bf16 [B,H,N,d], device, written.
+ *   lse         : fp32 [B,H,N], device, written (natural log).
+ * Other arguments and errors as fa_fwd; d != 128 gives FA_ERR_UNSUPPORTED_D.
+ */
+int fa_fwd_fp8(const void *q, const void *k, const void *v, const float *descale_q,
+               const float *descale_k, const float *descale_v, void *o, float *lse,
+               int B, int H, int N, int d, float scale, int causal, fa_stream_t stream);
+
+/*
  * Backward: gradients of L = sum(O * dO) for the forward above.  The
  * formulas are not on the pages (they only say the backward recomputes the
  * probabilities tile by tile); the library computes the exact gradient:
@@ -189,14 +211,40 @@ int fa_decode_plan(int BH, int Nq, int Nk, int d, int num_splits, int sms,
                    int ctas_per_sm, int *splits, int *chunk_keys);
 
 /*
+ * Matrix multiply C = A B: bf16 A [M,K] and B [K,N] (row-major with row
+ * strides lda, ldb), fp32 accumulation, bf16 C [M,N] (row stride ldc).  The
+ * matrix multiply of the throughput-versus-size curve that "CS336 Lecture 5 ·
+ * GPUs, TPUs" opens with (notes, opening goal and the "矩阵谜题" section):
+ * 256 x 128 output tiles, one persistent CTA per SM, so the tile count over
+ * the SM count sets the number of rounds (wave quantization).  An operand
+ * whose rows are not 16-byte aligned (leading dimension not a multiple of 8
+ * elements, or an unaligned base) is first copied into the workspace with an
+ * aligned leading dimension, because the tensor-memory copies need aligned
+ * rows; that copy is the cost of such sizes.
+ *   workspace : device scratch of fa_gemm_workspace_size(A, B, M, N, K, lda,
+ *               ldb) bytes (0 when both operands are aligned; NULL allowed
+ *               then), 16-byte aligned, owned by the caller.
+ * Pointers need only 2-byte alignment.  M, N, K >= 1, lda >= K, ldb >= N,
+ * ldc >= N.
+ */
+size_t fa_gemm_workspace_size(const void *A, const void *B, int M, int N, int K, int lda,
+                              int ldb);
+int fa_gemm(const void *A, const void *B, void *C, int M, int N, int K, int lda, int ldb,
+            int ldc, void *workspace, size_t workspace_bytes, fa_stream_t stream);
+
+/* Output tiles of fa_gemm: ceil(M / 256) x ceil(N / 128) (host arithmetic). */
+int fa_gemm_tiles(int M, int N, int *tiles_m, int *tiles_n);
+
+/*
  * Opt-in per-kernel timing with CUDA events (a tracing aid; off by default).
  * After fa_trace_start(), every kernel the library enqueues, on any stream of
  * any device, is bracketed by two CUDA events recorded on its launch stream,
  * until fa_trace_stop().  fa_trace_stop() waits for those events and fills,
  * for each kernel id k < n_kernels, launches[k] and total_ms[k] (summed event
  * durations).  Kernel ids: 0 forward, 1 backward preprocess, 2 backward main,
- * 3 dQ conversion, 4 dQ pass of the deterministic backward, 5 decode
- * (fa_trace_kernel_name gives the kernel's name).  The
+ * 3 dQ conversion, 4 dQ pass of the deterministic backward, 5 decode,
+ * 6 GEMM, 7 GEMM operand packing (fa_trace_kernel_name gives the kernel's
+ * name).  The
  * library creates the events on first use and reuses them afterwards; event
  * records add a few microseconds per launch.  fa_trace_start() discards a
  * previous unfinished record.

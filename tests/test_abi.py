@@ -128,3 +128,16 @@ def test_decode_plan(lib):
     assert fa.decode_plan(4, 8, 100000, 128, num_splits=1) == (196, 512)
     with pytest.raises(fa.FAError):
         fa.decode_plan(4, 9, 100, 128)
+
+
+# fa_fwd_fp8(q, k, v, dq, dk, dv, o, lse, B, H, N, d, scale, causal, stream)
+@pytest.mark.parametrize("args,code", [
+    ((P, P, P, 0, P, P, P, P, 1, 1, 16, 128, 0.1, 0, None), -1),      # NULL descale_q
+    ((P, P, P, P, P, P, P, P, 1, 1, 16, 64, 0.1, 0, None), -3),       # d = 64 (FP8 is d = 128)
+    ((P, P, P, P, P, P, P, P, 0, 1, 16, 128, 0.1, 0, None), -2),      # B = 0
+    ((P, P, P + 4, P, P, P, P, P, 1, 1, 16, 128, 0.1, 0, None), -4),  # misaligned v
+    ((P, P, P, P + 1, P, P, P, P, 1, 1, 16, 128, 0.1, 0, None), -4),  # misaligned descale
+    ((P, P, P, P, P, P, P, P, 1, 1, 16, 128, float("nan"), 0, None), -10),  # scale NaN
+])
+def test_fwd_fp8_validation(lib, args, code):
+    assert lib.fa_fwd_fp8(*args) == code

@@ -75,3 +75,22 @@ def test_sweep_has_48_cases():
     ws = inputs.sweep_workloads()
     assert len(ws) == 48
     assert len({w.name for w in ws}) == 48
+
+
+def test_fp8_input_recipe():
+    """fp8_qkv: per (b, h) the largest |x8| is the E4M3 maximum 448, and
+    x8 * descale reproduces the fp32 draws within E4M3 rounding (relative
+    2^-4 for normals, absolute 2^-10 * descale below the normal range)."""
+    import torch
+    q8, k8, v8, fq, fk, fv = inputs.fp8_qkv(2, 3, 200, 128, seed=4)
+    for x8 in (q8, k8, v8):
+        assert x8.dtype == torch.float8_e4m3fn and x8.shape == (2, 3, 200, 128)
+        assert torch.all(x8.float().abs().amax(dim=(2, 3)) == 448.0)
+    # the same fp32 draws as the bf16 recipe (bf16 rounding of both agrees to 2^-4)
+    q, k, v, _ = inputs.qkv_do(2, 3, 200, 128, seed=4)
+    for x8, f, ref in ((q8, fq, q), (k8, fk, k), (v8, fv, v)):
+        deq = x8.double() * f.double()[:, :, None, None]
+        r = ref.double()
+        tol = torch.maximum(2.0 ** -4 * r.abs() + 2.0 ** -8 * r.abs(),
+                            (2.0 ** -10) * f.double()[:, :, None, None])
+        assert torch.all((deq - r).abs() <= tol)

@@ -16,6 +16,7 @@
 #include "bwd_kernel.cuh"
 #include "decode_kernel.cuh"
 #include "dq_kernel.cuh"
+#include "gemm_kernel.cuh"
 #include "fwd_kernel.cuh"
 
 namespace {
@@ -46,10 +47,11 @@ EncodeTiledFn g_encode = nullptr;
 // Opt-in per-kernel timing: while enabled, every launch is bracketed by a
 // pair of CUDA events on its stream.
 enum { kKernFwd = 0, kKernBwdPrep = 1, kKernBwd = 2, kKernBwdConvert = 3, kKernDq = 4,
-       kKernDecode = 5, kNumKernels = 6 };
+       kKernDecode = 5, kKernGemm = 6, kKernGemmPack = 7, kNumKernels = 8 };
 const char* const kKernelNames[kNumKernels] = {"fa_fwd_kernel", "fa_bwd_prep", "fa_bwd_kernel",
                                                "fa_bwd_dq_convert", "fa_dq_kernel",
-                                               "fa_decode_kernel"};
+                                               "fa_decode_kernel", "fa_gemm_kernel",
+                                               "fa_gemm_pack"};
 struct TraceRec {
   int kernel;
   int device;
@@ -144,11 +146,11 @@ int make_tmap_rows(CUtensorMap* m, const void* base, int BH, int N, int d, int b
 
 int fwd_units(int B, int H, int N) { return B * H * ((N + 255) / 256); }
 
-template <int D, bool CAUSAL>
+template <int D, bool CAUSAL, bool FP8 = false>
 int launch_fwd(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                const fa::FwdParams& p, int ctas, cudaStream_t stream) {
-  auto kern = fa::fa_fwd_kernel<D, CAUSAL>;
-  const int smem = fa::FwdLayout<D>::kSmemBytes;
+  auto kern = fa::fa_fwd_kernel<D, CAUSAL, FP8>;
+  const int smem = fa::FwdLayout<D, FP8>::kSmemBytes;
   // The kernel moves registers between warpgroups; its split assumes the
   // launch allocation it was compiled for.  Refuse to launch otherwise
   // (a larger request than the block holds would never be granted).
@@ -173,6 +175,21 @@ int make_tmap_rows(CUtensorMap* m, const void* base, int BH, int N, int d, int b
   cuuint32_t box[3] = {64, static_cast<cuuint32_t>(box_rows), 1};
   cuuint32_t estr[3] = {1, 1, 1};
   CUresult r = g_encode(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims,
+                        strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                        CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                        CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? FA_OK : FA_ERR_LAUNCH;
+}
+
+// 3-D view [B*H][N][d] of an 8-bit tensor with d = 128: boxes of `box_rows`
+// rows x 128 columns (128 bytes, the 128-byte swizzle span).
+int make_tmap_rows_u8(CUtensorMap* m, const void* base, int BH, int N, int d, int box_rows) {
+  cuuint64_t dims[3] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(N),
+                        static_cast<cuuint64_t>(BH)};
+  cuuint64_t strides[2] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(N) * d};
+  cuuint32_t box[3] = {128, static_cast<cuuint32_t>(box_rows), 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = g_encode(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<void*>(base), dims,
                         strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
                         CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                         CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
@@ -443,6 +460,42 @@ int launch_decode(const fa::DecodeParams& p, int BH, int d, cudaStream_t stream)
   }
 }
 
+// ---------------------------------------------------------------- GEMM
+size_t gemm_ld8(int n) { return (static_cast<size_t>(n) + 7) / 8 * 8; }
+
+bool gemm_needs_pack(const void* ptr, int ld) {
+  return !aligned16(ptr) || (ld % 8) != 0;
+}
+
+size_t gemm_ws_bytes(const void* A, const void* B, int M, int N, int K, int lda, int ldb) {
+  size_t bytes = 0;
+  if (gemm_needs_pack(A, lda)) bytes += fa::round256(static_cast<size_t>(M) * gemm_ld8(K) * 2);
+  if (gemm_needs_pack(B, ldb)) bytes += fa::round256(static_cast<size_t>(K) * gemm_ld8(N) * 2);
+  return bytes;
+}
+
+// 2-D view [rows][cols] of a bf16 matrix with row stride `ld` elements
+// (a multiple of 8), boxes of box_rows x 64 columns, 128-byte swizzle.
+int make_tmap_2d(CUtensorMap* m, const void* base, int rows, int cols, int ld, int box_rows) {
+  cuuint64_t dims[2] = {static_cast<cuuint64_t>(cols), static_cast<cuuint64_t>(rows)};
+  cuuint64_t strides[1] = {static_cast<cuuint64_t>(ld) * 2};
+  cuuint32_t box[2] = {64, static_cast<cuuint32_t>(box_rows)};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = g_encode(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims,
+                        strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                        CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                        CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? FA_OK : FA_ERR_LAUNCH;
+}
+
+int launch_gemm_pack(const void* src, int ld_src, void* dst, int ld_dst, int rows, int cols,
+                     int sms, cudaStream_t stream) {
+  LaunchTrace trace(kKernGemmPack, stream);
+  fa::fa_gemm_pack<<<sms * 4, 256, 0, stream>>>(static_cast<const uint16_t*>(src), ld_src,
+                                                static_cast<uint16_t*>(dst), ld_dst, rows, cols);
+  return cudaPeekAtLastError() == cudaSuccess ? FA_OK : FA_ERR_LAUNCH;
+}
+
 // Split of a decode problem on the current device.
 int decode_device_plan(int B, int H, int Nq, int Nk, int d, int num_splits, DeviceInfo** info,
                        int* splits, int* chunk) {
@@ -578,6 +631,7 @@ int fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int
   fa::FwdParams p;
   p.o = static_cast<__nv_bfloat16*>(o);
   p.lse = lse;
+  p.descale_q = p.descale_k = p.descale_v = nullptr;
   p.BH = BH;
   p.N = N;
   p.n_qt2 = (N + 255) / 256;
@@ -594,6 +648,117 @@ int fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int
                   : launch_fwd<64, false>(tq, tk, tv, p, ctas, st);
   return causal ? launch_fwd<128, true>(tq, tk, tv, p, ctas, st)
                 : launch_fwd<128, false>(tq, tk, tv, p, ctas, st);
+}
+
+size_t fa_gemm_workspace_size(const void* A, const void* B, int M, int N, int K, int lda,
+                               int ldb) {
+  if (M < 1 || N < 1 || K < 1 || lda < K || ldb < N) return 0;
+  return gemm_ws_bytes(A, B, M, N, K, lda, ldb);
+}
+
+int fa_gemm_tiles(int M, int N, int* tiles_m, int* tiles_n) {
+  if (!tiles_m || !tiles_n) return FA_ERR_NULL;
+  if (M < 1 || N < 1) return FA_ERR_SHAPE;
+  *tiles_m = (M + fa::kGemmBM - 1) / fa::kGemmBM;
+  *tiles_n = (N + fa::kGemmBN - 1) / fa::kGemmBN;
+  return FA_OK;
+}
+
+int fa_gemm(const void* A, const void* B, void* C, int M, int N, int K, int lda, int ldb, int ldc,
+            void* workspace, size_t workspace_bytes, fa_stream_t stream) {
+  if (!A || !B || !C) return FA_ERR_NULL;
+  if (M < 1 || N < 1 || K < 1 || lda < K || ldb < N || ldc < N) return FA_ERR_SHAPE;
+  if (static_cast<long long>(M) * lda >= (1ll << 40) || static_cast<long long>(K) * ldb >= (1ll << 40) ||
+      static_cast<long long>(M) * ldc >= (1ll << 40))
+    return FA_ERR_SHAPE;
+  auto al2 = [](const void* ptr) { return (reinterpret_cast<uintptr_t>(ptr) & 1u) == 0; };
+  if (!al2(A) || !al2(B) || !al2(C)) return FA_ERR_ALIGN;
+  const size_t need = gemm_ws_bytes(A, B, M, N, K, lda, ldb);
+  if (need > 0) {
+    if (!workspace) return FA_ERR_NULL;
+    if (!aligned16(workspace)) return FA_ERR_ALIGN;
+    if (workspace_bytes < need) return FA_ERR_WORKSPACE;
+  }
+  DeviceInfo* info = nullptr;
+  int s = device_info(&info);
+  if (s != FA_OK) return s;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  // Operands whose rows are not 16-byte aligned go through an aligned copy.
+  const void* a_use = A;
+  const void* b_use = B;
+  int lda_use = lda, ldb_use = ldb;
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  if (gemm_needs_pack(A, lda)) {
+    lda_use = static_cast<int>(gemm_ld8(K));
+    if ((s = launch_gemm_pack(A, lda, ws, lda_use, M, K, info->sms, st)) != FA_OK) return s;
+    a_use = ws;
+    ws += fa::round256(static_cast<size_t>(M) * lda_use * 2);
+  }
+  if (gemm_needs_pack(B, ldb)) {
+    ldb_use = static_cast<int>(gemm_ld8(N));
+    if ((s = launch_gemm_pack(B, ldb, ws, ldb_use, K, N, info->sms, st)) != FA_OK) return s;
+    b_use = ws;
+  }
+  CUtensorMap ta, tb;
+  if (make_tmap_2d(&ta, a_use, M, K, lda_use, 128) != FA_OK ||
+      make_tmap_2d(&tb, b_use, K, N, ldb_use, 64) != FA_OK)
+    return FA_ERR_LAUNCH;
+  fa::GemmParams p;
+  p.c = static_cast<uint16_t*>(C);
+  p.M = M;
+  p.N = N;
+  p.K = K;
+  p.ldc = ldc;
+  p.tiles_n = (N + fa::kGemmBN - 1) / fa::kGemmBN;
+  p.n_tiles = ((M + fa::kGemmBM - 1) / fa::kGemmBM) * p.tiles_n;
+  p.k_blocks = (K + fa::kGemmBK - 1) / fa::kGemmBK;
+  p.status = info->status;
+  const int ctas = p.n_tiles < info->sms ? p.n_tiles : info->sms;
+  auto kern = fa::fa_gemm_kernel;
+  const int smem = fa::GemmLayout::kSmemBytes;
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
+    return FA_ERR_LAUNCH;
+  LaunchTrace trace(kKernGemm, st);
+  kern<<<ctas, 256, smem, st>>>(ta, tb, p);
+  return cudaPeekAtLastError() == cudaSuccess ? FA_OK : FA_ERR_LAUNCH;
+}
+
+int fa_fwd_fp8(const void* q, const void* k, const void* v, const float* descale_q,
+               const float* descale_k, const float* descale_v, void* o, float* lse, int B, int H,
+               int N, int d, float scale, int causal, fa_stream_t stream) {
+  if (!q || !k || !v || !descale_q || !descale_k || !descale_v || !o || !lse) return FA_ERR_NULL;
+  int s = check_shape(B, H, N, d);
+  if (s != FA_OK) return s;
+  if (d != 128) return FA_ERR_UNSUPPORTED_D;
+  if ((s = check_scale(scale)) != FA_OK) return s;
+  auto al4 = [](const void* ptr) { return (reinterpret_cast<uintptr_t>(ptr) & 3u) == 0; };
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(lse) ||
+      !al4(descale_q) || !al4(descale_k) || !al4(descale_v))
+    return FA_ERR_ALIGN;
+  DeviceInfo* info = nullptr;
+  if ((s = device_info(&info)) != FA_OK) return s;
+  const int BH = B * H;
+  CUtensorMap tq, tk, tv;
+  if (make_tmap_rows_u8(&tq, q, BH, N, d, 128) != FA_OK ||
+      make_tmap_rows_u8(&tk, k, BH, N, d, 128) != FA_OK ||
+      make_tmap_rows_u8(&tv, v, BH, N, d, 128) != FA_OK)
+    return FA_ERR_LAUNCH;
+  fa::FwdParams p;
+  p.o = static_cast<__nv_bfloat16*>(o);
+  p.lse = lse;
+  p.descale_q = descale_q;
+  p.descale_k = descale_k;
+  p.descale_v = descale_v;
+  p.BH = BH;
+  p.N = N;
+  p.n_qt2 = (N + 255) / 256;
+  p.n_units = fwd_units(B, H, N);
+  p.scale_log2 = scale * 1.4426950408889634f;  // the kernel folds in the descales, then clamps
+  p.status = info->status;
+  const int ctas = p.n_units < info->sms ? p.n_units : info->sms;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  return causal ? launch_fwd<128, true, true>(tq, tk, tv, p, ctas, st)
+                : launch_fwd<128, false, true>(tq, tk, tv, p, ctas, st);
 }
 
 int fa_bwd_deterministic(const void* q, const void* k, const void* v, const void* o,

@@ -31,7 +31,20 @@
 // only raised when a tile's maximum exceeds it by more than 2^8 (in the
 // exp2 domain), so most tiles skip the O read-modify-write.  The result is
 // unchanged because O and l are always scaled by the same reference.
+//
+// FP8 variant (FP8 = true, d = 128): Q, K and V arrive as E4M3 with one fp32
+// descale factor per head each (the low-precision operands of "第17讲" §4.4 /
+// "CS336 Lecture 5" on FP8).  S = Q K^T and O += P V run as kind::f8f6f4
+// MMAs (K = 32 per instruction, twice the bf16 rate); the score scale absorbs
+// descale_q * descale_k, P is stored to TMEM as E4M3 (4 per column) and the
+// output is O = descale_v * sum_j p~_j v_j / sum_j p~_j, where p~ is the E4M3
+// value of p actually used by the MMA, so O stays a convex combination of V
+// rows; lse uses the unrounded p.
 #pragma once
+#include <cfloat>
+#include <cuda_fp16.h>
+#include <cuda_fp8.h>
+
 #include "sm100.cuh"
 
 namespace fa {
@@ -39,6 +52,9 @@ namespace fa {
 struct FwdParams {
   __nv_bfloat16* o;
   float* lse;
+  const float* descale_q;  // FP8 only: per-head [B*H] dequantisation factors
+  const float* descale_k;
+  const float* descale_v;
   int BH;
   int N;
   int n_qt2;       // ceil(N / 256): Q tile pairs per head
@@ -47,10 +63,10 @@ struct FwdParams {
   int* status;
 };
 
-template <int D>
+template <int D, bool FP8 = false>
 struct FwdLayout {
-  static constexpr int kTileBytes = 128 * D * 2;
-  static constexpr int kStages = (D == 64) ? 4 : 2;
+  static constexpr int kTileBytes = 128 * D * (FP8 ? 1 : 2);
+  static constexpr int kStages = (FP8 || D == 64) ? 4 : 2;
   static constexpr int kQ0 = 0;
   static constexpr int kQ1 = kTileBytes;
   static constexpr int kK = 2 * kTileBytes;
@@ -120,7 +136,6 @@ __device__ __forceinline__ bool wait1(uint64_t* bar, uint32_t parity, FwdBarrier
 }
 
 // The same from every lane of a warp, with a warp-uniform answer.
-// The same from every lane of a warp, with a warp-uniform answer.
 __device__ __forceinline__ bool wait_warp(uint64_t* bar, uint32_t parity, FwdBarriers* b,
                                           int* status) {
   bool ok = !*(volatile int*)&b->abort_flag;
@@ -131,12 +146,15 @@ __device__ __forceinline__ bool wait_warp(uint64_t* bar, uint32_t parity, FwdBar
 }
 
 // ---------------------------------------------------------------- producer
-template <int D, bool CAUSAL>
+template <int D, bool CAUSAL, bool FP8>
 __device__ void fwd_producer(const CUtensorMap* tm_q, const CUtensorMap* tm_k,
                              const CUtensorMap* tm_v, const FwdParams& p, uint8_t* smem,
                              FwdBarriers* b, int& kc, int& vc, int& units) {
-  using L = FwdLayout<D>;
+  using L = FwdLayout<D, FP8>;
   constexpr int S = L::kStages;
+  // A tile is D/64 boxes of 64 bf16 columns, or one box of 128 E4M3 columns;
+  // either way a box row is 128 bytes.
+  constexpr int NB = FP8 ? 1 : D / 64;
   for (int r = 0, nr = snake_rounds(p.n_units); r < nr; ++r) {
     const int w = snake_unit(r, p.n_units);
     if (w < 0) continue;
@@ -145,7 +163,7 @@ __device__ void fwd_producer(const CUtensorMap* tm_q, const CUtensorMap* tm_k,
     mbar_arrive_expect_tx(&b->q_full, 2 * L::kTileBytes);
     ++units;  // number of times q_full has been armed
 #pragma unroll
-    for (int c = 0; c < D / 64; ++c) {
+    for (int c = 0; c < NB; ++c) {
       tma_load_3d(smem + L::kQ0 + c * 16384, tm_q, &b->q_full, c * 64, u.q0, u.bh);
       tma_load_3d(smem + L::kQ1 + c * 16384, tm_q, &b->q_full, c * 64, u.q0 + 128, u.bh);
     }
@@ -156,7 +174,7 @@ __device__ void fwd_producer(const CUtensorMap* tm_q, const CUtensorMap* tm_k,
         if (kc >= S && !wait1(&b->k_empty[st], ((kc / S) - 1) & 1, b, p.status)) return;
         mbar_arrive_expect_tx(&b->k_full[st], L::kTileBytes);
 #pragma unroll
-        for (int c = 0; c < D / 64; ++c)
+        for (int c = 0; c < NB; ++c)
           tma_load_3d(smem + L::kK + st * L::kTileBytes + c * 16384, tm_k, &b->k_full[st],
                       c * 64, j * 128, u.bh);
         ++kc;
@@ -166,7 +184,7 @@ __device__ void fwd_producer(const CUtensorMap* tm_q, const CUtensorMap* tm_k,
         if (vc >= S && !wait1(&b->v_empty[st], ((vc / S) - 1) & 1, b, p.status)) return;
         mbar_arrive_expect_tx(&b->v_full[st], L::kTileBytes);
 #pragma unroll
-        for (int c = 0; c < D / 64; ++c)
+        for (int c = 0; c < NB; ++c)
           tma_load_3d(smem + L::kV + st * L::kTileBytes + c * 16384, tm_v, &b->v_full[st],
                       c * 64, j * 128, u.bh);
         ++vc;
@@ -176,31 +194,52 @@ __device__ void fwd_producer(const CUtensorMap* tm_q, const CUtensorMap* tm_k,
 }
 
 // ---------------------------------------------------------------- MMA issuer
-template <int D>
+// S = Q K^T: K-major operands; each K-step reads the next 32 bytes of every
+// row (16 bf16 or 32 E4M3 elements), and a bf16 row of D > 64 continues in
+// the next 64-column box.
+template <int D, bool FP8>
 __device__ __forceinline__ void issue_s(uint32_t tmem_s, uint32_t q_smem, uint32_t k_smem) {
-  constexpr uint32_t idesc = idesc_bf16_f32(128, 128, false, false);
+  if constexpr (FP8) {
+    constexpr uint32_t idesc = idesc_e4m3_f32(128, 128, false, false);
 #pragma unroll
-  for (int kk = 0; kk < D / 16; ++kk) {
-    const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
-    mma_ss(tmem_s, sdesc_sw128(q_smem + off, 16, 1024), sdesc_sw128(k_smem + off, 16, 1024),
-           idesc, kk > 0 ? 1u : 0u);
+    for (int kk = 0; kk < D / 32; ++kk)
+      mma_ss_f8(tmem_s, sdesc_sw128(q_smem + kk * 32, 16, 1024),
+                sdesc_sw128(k_smem + kk * 32, 16, 1024), idesc, kk > 0 ? 1u : 0u);
+  } else {
+    constexpr uint32_t idesc = idesc_bf16_f32(128, 128, false, false);
+#pragma unroll
+    for (int kk = 0; kk < D / 16; ++kk) {
+      const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
+      mma_ss(tmem_s, sdesc_sw128(q_smem + off, 16, 1024), sdesc_sw128(k_smem + off, 16, 1024),
+             idesc, kk > 0 ? 1u : 0u);
+    }
   }
 }
 
-template <int D>
+// O += P V: A = P from TMEM (8 columns per K-step in both types: 16 bf16 or
+// 32 E4M3 keys), B = V MN-major (a K-step covers 16 or 32 key rows of 128
+// bytes; bf16 rows of D = 128 span two 64-column boxes 16 KB apart).
+template <int D, bool FP8>
 __device__ __forceinline__ void issue_pv(uint32_t tmem_o, uint32_t tmem_p, uint32_t v_smem,
                                          bool accumulate) {
-  constexpr uint32_t idesc = idesc_bf16_f32(128, D, false, true);
+  if constexpr (FP8) {
+    constexpr uint32_t idesc = idesc_e4m3_f32(128, D, false, true);
 #pragma unroll
-  for (int kk = 0; kk < 8; ++kk) {
-    mma_ts(tmem_o, tmem_p + kk * 8, sdesc_sw128(v_smem + kk * 2048, 16384, 1024), idesc,
-           (accumulate || kk > 0) ? 1u : 0u);
+    for (int kk = 0; kk < 4; ++kk)
+      mma_ts_f8(tmem_o, tmem_p + kk * 8, sdesc_sw128(v_smem + kk * 4096, 16384, 1024), idesc,
+                (accumulate || kk > 0) ? 1u : 0u);
+  } else {
+    constexpr uint32_t idesc = idesc_bf16_f32(128, D, false, true);
+#pragma unroll
+    for (int kk = 0; kk < 8; ++kk)
+      mma_ts(tmem_o, tmem_p + kk * 8, sdesc_sw128(v_smem + kk * 2048, 16384, 1024), idesc,
+             (accumulate || kk > 0) ? 1u : 0u);
   }
 }
 
-template <int D, bool CAUSAL>
+template <int D, bool CAUSAL, bool FP8>
 __device__ void fwd_mma(const FwdParams& p, uint8_t* smem, FwdBarriers* b, uint32_t tmem) {
-  using L = FwdLayout<D>;
+  using L = FwdLayout<D, FP8>;
   constexpr int S = L::kStages;
   const uint32_t sb = smem_u32(smem);
   const uint32_t tS[2] = {tmem + 0, tmem + 128};
@@ -231,18 +270,18 @@ __device__ void fwd_mma(const FwdParams& p, uint8_t* smem, FwdBarriers* b, uint3
         if (!wait1(&b->p_full[0], pc[0] & 1, b, p.status)) return;
         ++pc[0];
         tc_fence_after();
-        issue_pv<D>(tO[0], tS[0], v_smem, j - 1 > 0);
+        issue_pv<D, FP8>(tO[0], tS[0], v_smem, j - 1 > 0);
         if (j - 1 == nk0 - 1) mma_commit(&b->o_full[0]);
       }
       if (j < nk0) {
-        issue_s<D>(tS[0], qs[0], k_smem);
+        issue_s<D, FP8>(tS[0], qs[0], k_smem);
         mma_commit(&b->s_full[0]);
       }
       if (j >= 1 && j - 1 < nk1) {
         if (!wait1(&b->p_full[1], pc[1] & 1, b, p.status)) return;
         ++pc[1];
         tc_fence_after();
-        issue_pv<D>(tO[1], tS[1], v_smem, j - 1 > 0);
+        issue_pv<D, FP8>(tO[1], tS[1], v_smem, j - 1 > 0);
         if (j - 1 == nk1 - 1) mma_commit(&b->o_full[1]);
       }
       if (j >= 1) {
@@ -250,7 +289,7 @@ __device__ void fwd_mma(const FwdParams& p, uint8_t* smem, FwdBarriers* b, uint3
         ++vc;
       }
       if (j < nk1) {
-        issue_s<D>(tS[1], qs[1], k_smem);
+        issue_s<D, FP8>(tS[1], qs[1], k_smem);
         mma_commit(&b->s_full[1]);
       }
       mma_commit(&b->k_empty[ks]);
@@ -266,14 +305,14 @@ __device__ void fwd_mma(const FwdParams& p, uint8_t* smem, FwdBarriers* b, uint3
       if (!wait1(&b->p_full[0], pc[0] & 1, b, p.status)) return;
       ++pc[0];
       tc_fence_after();
-      issue_pv<D>(tO[0], tS[0], v_smem, nk - 1 > 0);
+      issue_pv<D, FP8>(tO[0], tS[0], v_smem, nk - 1 > 0);
       mma_commit(&b->o_full[0]);
     }
     if (nk - 1 < nk1) {
       if (!wait1(&b->p_full[1], pc[1] & 1, b, p.status)) return;
       ++pc[1];
       tc_fence_after();
-      issue_pv<D>(tO[1], tS[1], v_smem, nk - 1 > 0);
+      issue_pv<D, FP8>(tO[1], tS[1], v_smem, nk - 1 > 0);
       mma_commit(&b->o_full[1]);
     }
     mma_commit(&b->v_empty[vs]);
@@ -282,13 +321,64 @@ __device__ void fwd_mma(const FwdParams& p, uint8_t* smem, FwdBarriers* b, uint3
 }
 
 // ---------------------------------------------------------------- softmax
-template <int D, bool CAUSAL>
+// Two probabilities as E4M3 (x.x in the low byte), and that pair back as f16.
+__device__ __forceinline__ uint32_t pack_e4m3x2(float2 x) {
+  return static_cast<uint32_t>(__nv_cvt_float2_to_fp8x2(x, __NV_SATFINITE, __NV_E4M3));
+}
+__device__ __forceinline__ __half2 e4m3x2_to_half2(uint32_t v) {
+  return __half2(__nv_cvt_fp8x2_to_halfraw2(static_cast<__nv_fp8x2_storage_t>(v), __NV_E4M3));
+}
+
+// FP8: P of one 128-key tile as E4M3, four keys per TMEM column (16 columns
+// per half of 64 keys).  Adds the unrounded p to rs (for lse) and returns the
+// sum of the rounded p (O's normaliser), accumulated in f16 pairs over 8
+// pairs and then in fp32.  Masked tiles use the MUFU exp2 throughout so that
+// masked probabilities are exactly 0; others take the polynomial on 3 of
+// every 8 pairs.
+template <bool MASKED>
+__device__ __forceinline__ float fp8_p_tile(const float* s, float2 sl2v, float2 nmb, float2* rs,
+                                            uint32_t tS) {
+  float lq = 0.f;
+#pragma unroll
+  for (int h = 0; h < 2; ++h) {
+    uint32_t pk[16];
+    __half2 hq[4] = {__float2half2_rn(0.f), __float2half2_rn(0.f), __float2half2_rn(0.f),
+                     __float2half2_rn(0.f)};
+#pragma unroll
+    for (int q4 = 0; q4 < 16; ++q4) {
+      const int c = 64 * h + 4 * q4;
+      const float2 xa = fma2(make_float2(s[c], s[c + 1]), sl2v, nmb);
+      const float2 xb = fma2(make_float2(s[c + 2], s[c + 3]), sl2v, nmb);
+      const int qa = 2 * q4, qb = 2 * q4 + 1;
+      float2 pa, pb;
+      if (!MASKED && (qa & 7) < 3)
+        pa = exp2_poly2(xa);
+      else
+        pa = make_float2(ex2_approx(xa.x), ex2_approx(xa.y));
+      if (!MASKED && (qb & 7) < 3)
+        pb = exp2_poly2(xb);
+      else
+        pb = make_float2(ex2_approx(xb.x), ex2_approx(xb.y));
+      rs[qa & 3] = add2(rs[qa & 3], pa);
+      rs[qb & 3] = add2(rs[qb & 3], pb);
+      const uint32_t ea = pack_e4m3x2(pa), eb = pack_e4m3x2(pb);
+      pk[q4] = ea | (eb << 16);
+      hq[q4 & 3] = __hadd2(hq[q4 & 3], __hadd2(e4m3x2_to_half2(ea), e4m3x2_to_half2(eb)));
+    }
+    tmem_st_x16(tS + 16 * h, pk);
+    const float2 f = __half22float2(__hadd2(hq[0], hq[1]));
+    const float2 g = __half22float2(__hadd2(hq[2], hq[3]));
+    lq += (f.x + f.y) + (g.x + g.y);
+  }
+  return lq;
+}
+
+template <int D, bool CAUSAL, bool FP8>
 __device__ void fwd_softmax(const FwdParams& p, FwdBarriers* b, uint32_t tmem, int wg) {
   const int t = threadIdx.x - 128 * (wg + 1);  // row within the Q tile == TMEM lane
   const uint32_t lane_base = static_cast<uint32_t>(t & ~31) << 16;
   const uint32_t tS = tmem + lane_base + (wg ? 128u : 0u);
   const uint32_t tO = tmem + lane_base + 256u + wg * D;
-  const float sl2 = p.scale_log2;
   const int N = p.N;
   int sc = 0, oc = 0;
   for (int r = 0, nr = snake_rounds(p.n_units); r < nr; ++r) {
@@ -298,8 +388,13 @@ __device__ void fwd_softmax(const FwdParams& p, FwdBarriers* b, uint32_t tmem, i
     const int nk = wg ? u.nk1 : u.nk0;
     const int tile_row0 = u.q0 + wg * 128;
     const int row = tile_row0 + t;
+    // FP8: the scores of E4M3 Q and K carry the two per-head descale factors.
+    const float sl2 = FP8 ? fmaxf(p.scale_log2 * __ldg(p.descale_q + u.bh) *
+                                      __ldg(p.descale_k + u.bh), FLT_MIN)
+                          : p.scale_log2;
     float m_used = -INFINITY;  // reference max (exp2 domain) of O and l
     float l = 0.f;
+    float lq = 0.f;  // FP8: sum of the E4M3-rounded p (O's normaliser)
     for (int j = 0; j < nk; ++j) {
       if (!wait_warp(&b->s_full[wg], sc & 1, b, p.status)) return;
       ++sc;
@@ -329,6 +424,7 @@ __device__ void fwd_softmax(const FwdParams& p, FwdBarriers* b, uint32_t tmem, i
         const float m_new = fmaxf(m_used, m_tile);
         const float alpha = (m_new == -INFINITY) ? 1.f : ex2_approx(m_used - m_new);
         l *= alpha;
+        lq *= alpha;
         if (j > 0) {
 #pragma unroll
           for (int c0 = 0; c0 < D; c0 += 16) {
@@ -351,7 +447,12 @@ __device__ void fwd_softmax(const FwdParams& p, FwdBarriers* b, uint32_t tmem, i
       // unmasked tiles 3 of every 8 pairs take the polynomial exp2 on the
       // FMA pipe and the rest the MUFU unit; masked tiles (which hold -inf)
       // use the MUFU unit throughout so masked probabilities are exactly 0.
-      if (need_mask) {
+      if constexpr (FP8) {
+        if (need_mask)
+          lq += fp8_p_tile<true>(s, sl2v, nmb, rs, tS);
+        else
+          lq += fp8_p_tile<false>(s, sl2v, nmb, rs, tS);
+      } else if (need_mask) {
 #pragma unroll
         for (int h = 0; h < 2; ++h) {
           uint32_t pk[32];
@@ -392,7 +493,8 @@ __device__ void fwd_softmax(const FwdParams& p, FwdBarriers* b, uint32_t tmem, i
     if (!wait_warp(&b->o_full[wg], oc & 1, b, p.status)) return;
     ++oc;
     tc_fence_after();
-    const float inv_l = 1.f / l;
+    // FP8: O = descale_v * (sum p~ v) / (sum p~).
+    const float inv_l = FP8 ? __ldg(p.descale_v + u.bh) / lq : 1.f / l;
     const bool valid = row < N;
     __nv_bfloat16* orow = p.o + (static_cast<size_t>(u.bh) * N + row) * D;
     uint32_t o[D];
@@ -415,11 +517,11 @@ __device__ void fwd_softmax(const FwdParams& p, FwdBarriers* b, uint32_t tmem, i
 }
 
 // ---------------------------------------------------------------- kernel
-template <int D, bool CAUSAL>
+template <int D, bool CAUSAL, bool FP8 = false>
 __global__ void __launch_bounds__(384, 1)
     fa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                   const __grid_constant__ CUtensorMap tm_v, const FwdParams p) {
-  using L = FwdLayout<D>;
+  using L = FwdLayout<D, FP8>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
@@ -460,13 +562,13 @@ __global__ void __launch_bounds__(384, 1)
   if (warp >= 4) {
     // Softmax warpgroups: take the registers warpgroup 0 gives up.
     regs_increase<kFwdSoftmaxRegs>();
-    fwd_softmax<D, CAUSAL>(p, b, tmem, (warp - 4) >> 2);
+    fwd_softmax<D, CAUSAL, FP8>(p, b, tmem, (warp - 4) >> 2);
   } else {
     regs_decrease<kFwdCtlRegs>();
     if (warp == 0) {
       if (lane_id() == 0) {
         int kc = 0, vc = 0, units = 0;
-        fwd_producer<D, CAUSAL>(&tm_q, &tm_k, &tm_v, p, smem, b, kc, vc, units);
+        fwd_producer<D, CAUSAL, FP8>(&tm_q, &tm_k, &tm_v, p, smem, b, kc, vc, units);
         // Wait for every TMA load this thread armed (all long complete on the
         // normal path) so no copy is in flight when the CTA exits.
         constexpr int S = L::kStages;
@@ -481,7 +583,7 @@ __global__ void __launch_bounds__(384, 1)
       __syncwarp();
     } else if (warp == 1) {
       if (lane_id() == 0) {
-        fwd_mma<D, CAUSAL>(p, smem, b, tmem);
+        fwd_mma<D, CAUSAL, FP8>(p, smem, b, tmem);
         // Drain every MMA this thread issued before TMEM is released.
         mma_commit(&b->mma_done);
         mbar_wait(&b->mma_done, 0, p.status);

@@ -28,10 +28,11 @@ STATUS_NAMES = {
 EXPORTED = ["fa_fwd", "fa_bwd", "fa_bwd_workspace_size", "fa_strerror",
             "fa_check_device_errors", "fa_launch_shape", "fa_trace_start", "fa_trace_stop",
             "fa_trace_kernel_name", "fa_bwd_noalloc", "fa_bwd_deterministic",
-            "fa_decode", "fa_decode_workspace_size", "fa_decode_plan"]
+            "fa_decode", "fa_decode_workspace_size", "fa_decode_plan", "fa_fwd_fp8",
+            "fa_gemm", "fa_gemm_workspace_size", "fa_gemm_tiles"]
 NOALLOC_MAX_SCRATCH = 32 << 20  # FA_BWD_NOALLOC_MAX_SCRATCH
 KERNEL_IDS = {0: "fa_fwd_kernel", 1: "fa_bwd_prep", 2: "fa_bwd_kernel", 3: "fa_bwd_dq_convert",
-              4: "fa_dq_kernel", 5: "fa_decode_kernel"}
+              4: "fa_dq_kernel", 5: "fa_decode_kernel", 6: "fa_gemm_kernel", 7: "fa_gemm_pack"}
 DECODE_MAX_NQ = 8
 
 
@@ -79,6 +80,15 @@ def load(path: str = LIB_PATH):
         lib.fa_bwd_noalloc.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp,
                                        _i, _i, _i, _i, _f, _i, _i, _vp]
         lib.fa_bwd_noalloc.restype = _i
+        lib.fa_gemm.argtypes = [_vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _vp, _sz, _vp]
+        lib.fa_gemm.restype = _i
+        lib.fa_gemm_workspace_size.argtypes = [_vp, _vp, _i, _i, _i, _i, _i]
+        lib.fa_gemm_workspace_size.restype = _sz
+        lib.fa_gemm_tiles.argtypes = [_i, _i, ctypes.POINTER(_i), ctypes.POINTER(_i)]
+        lib.fa_gemm_tiles.restype = _i
+        lib.fa_fwd_fp8.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _f,
+                                   _i, _vp]
+        lib.fa_fwd_fp8.restype = _i
         lib.fa_decode.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _f, _i,
                                   _i, _vp, _sz, _vp]
         lib.fa_decode.restype = _i
@@ -138,6 +148,37 @@ def fwd(q, k, v, scale=None, causal=False, out=None, lse=None):
         st = load().fa_fwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(),
                            lse.data_ptr(), B, H, N, d, scale, int(bool(causal)), _stream(q.device))
     _check(st, "fa_fwd")
+    return out, lse
+
+
+def fwd_fp8(q, k, v, descale_q, descale_k, descale_v, scale=None, causal=False, out=None,
+            lse=None):
+    """fa_fwd_fp8: q, k, v are float8_e4m3fn [B,H,N,128] CUDA tensors and
+    descale_* fp32 [B,H] per-head dequantisation factors.  Returns O bf16
+    [B,H,N,128] and lse fp32 [B,H,N]."""
+    if q.dim() != 4:
+        raise ValueError("expected [B, H, N, d] tensors")
+    for t in (q, k, v):
+        if not t.is_cuda or t.dtype != torch.float8_e4m3fn or not t.is_contiguous():
+            raise ValueError("q, k, v must be contiguous float8_e4m3fn CUDA tensors")
+        if t.shape != q.shape or t.device != q.device:
+            raise ValueError("q, k, v must share shape and device")
+    B, H, N, d = q.shape
+    for t in (descale_q, descale_k, descale_v):
+        if (not t.is_cuda or t.dtype != torch.float32 or t.numel() != B * H
+                or not t.is_contiguous()):
+            raise ValueError("descale factors must be contiguous fp32 [B, H] CUDA tensors")
+    scale = default_scale(d) if scale is None else float(scale)
+    if out is None:
+        out = torch.empty(q.shape, dtype=torch.bfloat16, device=q.device)
+    if lse is None:
+        lse = torch.empty((B, H, N), dtype=torch.float32, device=q.device)
+    with torch.cuda.device(q.device):
+        st = load().fa_fwd_fp8(q.data_ptr(), k.data_ptr(), v.data_ptr(), descale_q.data_ptr(),
+                               descale_k.data_ptr(), descale_v.data_ptr(), out.data_ptr(),
+                               lse.data_ptr(), B, H, N, d, scale, int(bool(causal)),
+                               _stream(q.device))
+    _check(st, "fa_fwd_fp8")
     return out, lse
 
 
@@ -278,3 +319,40 @@ def decode(q, k_cache, v_cache, cache_lens=None, scale=None, causal=False, nk=No
                               workspace.data_ptr(), workspace.numel(), _stream(q.device))
     _check(st, "fa_decode")
     return out, lse
+
+
+def gemm_tiles(M, N):
+    """(tiles_m, tiles_n) of fa_gemm's 256 x 128 output tiles."""
+    tm, tn = _i(0), _i(0)
+    _check(load().fa_gemm_tiles(M, N, ctypes.byref(tm), ctypes.byref(tn)), "fa_gemm_tiles")
+    return tm.value, tn.value
+
+
+def _ld(t):
+    if t.dim() != 2 or t.stride(1) != 1 or t.stride(0) < t.shape[1]:
+        raise ValueError("expected a 2-D matrix with unit column stride (rows may be padded)")
+    return t.stride(0)
+
+
+def gemm(a, b, out=None, workspace=None):
+    """fa_gemm: C = A B for bf16 CUDA matrices A [M, K], B [K, N] (rows may be
+    strided).  Returns C bf16 [M, N]."""
+    for t in (a, b):
+        if not t.is_cuda or t.dtype != torch.bfloat16:
+            raise ValueError("A and B must be bf16 CUDA matrices")
+    M, K = a.shape
+    K2, N = b.shape
+    if K2 != K or b.device != a.device:
+        raise ValueError("A [M, K] and B [K, N] on one device")
+    lda, ldb = _ld(a), _ld(b)
+    if out is None:
+        out = torch.empty((M, N), dtype=torch.bfloat16, device=a.device)
+    ldc = _ld(out)
+    with torch.cuda.device(a.device):
+        need = int(load().fa_gemm_workspace_size(a.data_ptr(), b.data_ptr(), M, N, K, lda, ldb))
+        if workspace is None or workspace.numel() < need:
+            workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=a.device)
+        st = load().fa_gemm(a.data_ptr(), b.data_ptr(), out.data_ptr(), M, N, K, lda, ldb, ldc,
+                            workspace.data_ptr(), workspace.numel(), _stream(a.device))
+    _check(st, "fa_gemm")
+    return out

@@ -15,6 +15,11 @@ Recipe (one generator per call, seeded with ``seed``):
    keep standard deviation 1.
 3. Everything is rounded to bf16 (round to nearest even).
 
+FP8 inputs (``fp8_qkv``): the fp32 draws of steps 1-2 (before any bf16
+rounding), then per (b, h) and per tensor a dequantisation factor
+amax / 448 (448 is the largest E4M3 value; 1 for an all-zero head) and the
+E4M3 value of x / factor (``torch.float8_e4m3fn``, round to nearest even).
+
 Decode inputs (``decode_qkv``): one generator per call; ``torch.randn`` fp32
 for q [B, H, Nq, d], then the caches k, v [B, H, L, d]; with ``ragged`` the
 per-batch valid lengths are then drawn uniformly from [L/2, L] with
@@ -103,9 +108,28 @@ def sweep_workloads():
     return out
 
 
+def fp8_qkv(B: int, H: int, N: int, d: int, seed: int = 0, dist: str = "normal"):
+    """(q8, k8, v8, descale_q, descale_k, descale_v): float8_e4m3fn
+    [B, H, N, d] tensors and fp32 [B, H] factors with x ~ x8 * factor."""
+    q, k, v, _ = _draw_fp32(B, H, N, d, seed, dist)
+    out8, scales = [], []
+    for x in (q, k, v):
+        amax = x.abs().amax(dim=(2, 3))
+        f = torch.where(amax > 0, amax / 448.0, torch.ones_like(amax)).to(torch.float32)
+        out8.append((x / f[:, :, None, None]).to(torch.float8_e4m3fn).contiguous())
+        scales.append(f.contiguous())
+    return (*out8, *scales)
+
+
 def qkv_do(B: int, H: int, N: int, d: int, seed: int = 0, dist: str = "normal",
            device: str | torch.device = "cpu"):
     """(q, k, v, dO) as contiguous bf16 [B, H, N, d] tensors."""
+    q, k, v, dO = _draw_fp32(B, H, N, d, seed, dist)
+    return tuple(t.to(torch.bfloat16).contiguous().to(device) for t in (q, k, v, dO))
+
+
+def _draw_fp32(B: int, H: int, N: int, d: int, seed: int, dist: str):
+    """Steps 1-2 of the recipe: the fp32 draws before rounding."""
     g = torch.Generator(device="cpu").manual_seed(int(seed))
     shape = (B, H, N, d)
     q = torch.randn(shape, generator=g, dtype=torch.float32)
@@ -124,10 +148,7 @@ def qkv_do(B: int, H: int, N: int, d: int, seed: int = 0, dist: str = "normal",
                 k[b, h, ik] *= 8.0
     elif dist != "normal":
         raise ValueError(f"unknown distribution {dist!r}")
-    out = tuple(t.to(torch.bfloat16).contiguous() for t in (q, k, v, dO))
-    if str(device) != "cpu":
-        out = tuple(t.to(device) for t in out)
-    return out
+    return q, k, v, dO
 
 
 def for_workload(w: Workload, device="cpu"):
