@@ -80,6 +80,9 @@ def parse_args():
                     help="time fa_bwd_deterministic (bit-reproducible dQ) instead of fa_bwd")
     ap.add_argument("--gemm-sweep", action="store_true",
                     help="time fa_gemm on square sizes of every divisibility class instead")
+    ap.add_argument("--gemm-sizes", default=None,
+                    help="comma-separated square sizes for --gemm-sweep (default: the full "
+                         "sweep); the value is taken at the largest")
     ap.add_argument("--fp8", action="store_true",
                     help="time fa_fwd_fp8 (E4M3 operands) on the benchmark shape instead")
     ap.add_argument("--decode", default=None, metavar="WORKLOAD",
@@ -480,7 +483,8 @@ def run_gemm_sweep(args, rank, world, local_rank, dist):
     sampler.start()
     time.sleep(0.4)
     sweep = []
-    sizes = [256 * i + dlt for i in range(1, 33) for dlt in (0, 1, 2, 8, 16)]
+    sizes = ([int(x) for x in args.gemm_sizes.split(",")] if args.gemm_sizes else
+             [256 * i + dlt for i in range(1, 33) for dlt in (0, 1, 2, 8, 16)])
     launches = 0
     for n in sizes:
         a = torch.randn((n, n), generator=g, device=dev, dtype=torch.float32).to(torch.bfloat16)
@@ -496,16 +500,16 @@ def run_gemm_sweep(args, rank, world, local_rank, dist):
                       "cublas_tflops": fl / ms_cublas / 1e9})
     clocks = sampler.stop()
     fa.check_device_errors(dev)
-    top = next(r for r in sweep if r["N"] == 8192)
+    top = next((r for r in sweep if r["N"] == 8192), max(sweep, key=lambda r: r["N"]))
     value = top["tflops"] * world
     roof = {"bound": "tensor", "achieved": top["tflops"], "peak": peaks["bf16_tflops"],
             "unit": "TFLOP/s", "frac": top["tflops"] / peaks["bf16_tflops"], "traffic": None,
             "kernel": "fa_gemm_kernel", "peak_source": f"{peaks_src} bf16_tflops (burst)",
-            "launch_ms": top["ms"], "at": "N=8192"}
+            "launch_ms": top["ms"], "at": f"N={top['N']}"}
 
     e2e = None
     if not args.no_e2e:
-        n = 8192
+        n = top["N"]
         ha = torch.randn((n, n), generator=torch.Generator().manual_seed(1)).to(torch.bfloat16).pin_memory()
         hb = torch.randn((n, n), generator=torch.Generator().manual_seed(2)).to(torch.bfloat16).pin_memory()
         hc = torch.empty((n, n), dtype=torch.bfloat16).pin_memory()
@@ -555,7 +559,9 @@ def run_gemm_sweep(args, rank, world, local_rank, dist):
             "steps": reps, "warmup": args.warmup, "ms_per_step": top["ms"],
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
             "dtype": "bf16", "data": "synthetic",
-            "config": {"workload": "gemm_square_sweep_N256_to_8208", "value_at": "N=8192",
+            "config": {"workload": ("gemm_square_sweep_N256_to_8208" if not args.gemm_sizes
+                                    else "gemm_square_" + args.gemm_sizes.replace(",", "_")),
+                       "value_at": f"N={top['N']}",
                        "tile": "256x128", "sms": sms, "l2": "flushed before every timed launch",
                        "parallelism": f"replicated per GPU x{world}"},
             "pct_of_peak": top["tflops"] / peaks["bf16_tflops"],
@@ -626,7 +632,8 @@ def run_fp8(args, rank, world, local_rank, dist):
     peak8 = 2.0 * peaks["bf16_tflops"]  # nominal dense fp8 / bf16 ratio: 4.5 / 2.25
     achieved = flops / (launch_ms * 1e-3) / 1e12
     roof = {"bound": "tensor", "achieved": achieved, "peak": peak8, "unit": "TFLOP/s",
-            "frac": achieved / peak8, "traffic": None, "kernel": "fa_fwd_kernel (fp8)",
+            "frac": achieved / peak8, "traffic": profiled_traffic("fa_fwd_kernel:fp8"),
+            "kernel": "fa_fwd_kernel (fp8)",
             "peak_source": f"{peaks_src} bf16_tflops (burst) x 2, the nominal fp8/bf16 ratio",
             "launch_ms": launch_ms}
     kernels = {name: {"launches": n, "avg_ms": t / n} for name, (n, t) in traced.items()}
