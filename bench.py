@@ -61,7 +61,8 @@ UNIT = "TFLOP/s"
 # The source file that defines each profiled kernel: a committed DRAM-traffic
 # figure stays valid while that file is unchanged.
 KERNEL_SOURCES = {"fa_fwd_kernel": "fwd_kernel.cuh", "fa_bwd_kernel": "bwd_kernel.cuh",
-                  "fa_dq_kernel": "dq_kernel.cuh", "fa_decode_kernel": "decode_kernel.cuh"}
+                  "fa_dq_kernel": "dq_kernel.cuh", "fa_decode_kernel": "decode_kernel.cuh",
+                  "fa_gemm_kernel": "gemm_kernel.cuh"}
 
 
 def parse_args():
@@ -492,10 +493,10 @@ def run_gemm_sweep(args, rank, world, local_rank, dist):
         c = torch.empty((n, n), dtype=torch.bfloat16, device=dev)
         ms = timed(lambda: fa.gemm(a, b, out=c, workspace=ws))
         ms_cublas = timed(lambda: torch.matmul(a, b, out=c))
-        tm, tn = fa.gemm_tiles(n, n)
+        bn, tm, tn = fa.gemm_tiles(n, n, sms)
         launches += (n_warm + reps) * (1 if n % 8 == 0 else 3)  # GEMM (+ two aligned copies)
         fl = 2.0 * n * n * n
-        sweep.append({"N": n, "div": gemm_div_class(n), "tiles": tm * tn,
+        sweep.append({"N": n, "div": gemm_div_class(n), "tile": f"256x{bn}", "tiles": tm * tn,
                       "rounds": -(-(tm * tn) // sms), "ms": ms, "tflops": fl / ms / 1e9,
                       "cublas_tflops": fl / ms_cublas / 1e9})
     clocks = sampler.stop()
@@ -503,7 +504,8 @@ def run_gemm_sweep(args, rank, world, local_rank, dist):
     top = next((r for r in sweep if r["N"] == 8192), max(sweep, key=lambda r: r["N"]))
     value = top["tflops"] * world
     roof = {"bound": "tensor", "achieved": top["tflops"], "peak": peaks["bf16_tflops"],
-            "unit": "TFLOP/s", "frac": top["tflops"] / peaks["bf16_tflops"], "traffic": None,
+            "unit": "TFLOP/s", "frac": top["tflops"] / peaks["bf16_tflops"],
+            "traffic": profiled_traffic(f"fa_gemm_kernel:{top['N']}"),
             "kernel": "fa_gemm_kernel", "peak_source": f"{peaks_src} bf16_tflops (burst)",
             "launch_ms": top["ms"], "at": f"N={top['N']}"}
 
@@ -562,7 +564,8 @@ def run_gemm_sweep(args, rank, world, local_rank, dist):
             "config": {"workload": ("gemm_square_sweep_N256_to_8208" if not args.gemm_sizes
                                     else "gemm_square_" + args.gemm_sizes.replace(",", "_")),
                        "value_at": f"N={top['N']}",
-                       "tile": "256x128", "sms": sms, "l2": "flushed before every timed launch",
+                       "tile": "256x256 when that fills the SMs, else 256x128", "sms": sms,
+                       "l2": "flushed before every timed launch",
                        "parallelism": f"replicated per GPU x{world}"},
             "pct_of_peak": top["tflops"] / peaks["bf16_tflops"],
             "roofline": roof, "cpu_baseline": cpu, "e2e": e2e,

@@ -215,8 +215,9 @@ int fa_decode_plan(int BH, int Nq, int Nk, int d, int num_splits, int sms,
  * strides lda, ldb), fp32 accumulation, bf16 C [M,N] (row stride ldc).  The
  * matrix multiply of the throughput-versus-size curve that "CS336 Lecture 5 ·
  * GPUs, TPUs" opens with (notes, opening goal and the "矩阵谜题" section):
- * 256 x 128 output tiles, one persistent CTA per SM, so the tile count over
- * the SM count sets the number of rounds (wave quantization).  An operand
+ * 256 x 128 or 256 x 256 output tiles (fa_gemm_tiles), one persistent CTA per
+ * SM, so the tile count over the SM count sets the number of rounds (wave
+ * quantization).  An operand
  * whose rows are not 16-byte aligned (leading dimension not a multiple of 8
  * elements, or an unaligned base) is first copied into the workspace with an
  * aligned leading dimension, because the tensor-memory copies need aligned
@@ -232,8 +233,10 @@ size_t fa_gemm_workspace_size(const void *A, const void *B, int M, int N, int K,
 int fa_gemm(const void *A, const void *B, void *C, int M, int N, int K, int lda, int ldb,
             int ldc, void *workspace, size_t workspace_bytes, fa_stream_t stream);
 
-/* Output tiles of fa_gemm: ceil(M / 256) x ceil(N / 128) (host arithmetic). */
-int fa_gemm_tiles(int M, int N, int *tiles_m, int *tiles_n);
+/* Output tiling of fa_gemm on a device with `sms` SMs (host arithmetic):
+ * tiles are 256 x *tile_n, *tile_n = 256 when ceil(M/256) x ceil(N/256) >= sms
+ * (every SM still gets a tile), else 128; *tiles_m x *tiles_n of them. */
+int fa_gemm_tiles(int M, int N, int sms, int *tile_n, int *tiles_m, int *tiles_n);
 
 /*
  * Opt-in per-kernel timing with CUDA events (a tracing aid; off by default).

@@ -141,3 +141,16 @@ def test_decode_plan(lib):
 ])
 def test_fwd_fp8_validation(lib, args, code):
     assert lib.fa_fwd_fp8(*args) == code
+
+
+def test_gemm_tiles(lib):
+    """Tile width 256 once a 256-wide tiling still covers every SM, else 128;
+    the lecture's 1792 -> 1793 example in 256 x 128 tiles is 98 -> 120 tiles."""
+    import tiled_attention_20_b200.fa as fa
+    assert fa.gemm_tiles(1792, 1792, 108) == (128, 7, 14)    # 98 tiles
+    assert fa.gemm_tiles(1793, 1793, 108) == (128, 8, 15)    # 120 tiles
+    assert fa.gemm_tiles(8192, 8192, 148) == (256, 32, 32)   # 1024 >= 148
+    assert fa.gemm_tiles(2048, 2048, 148) == (128, 8, 16)    # 64 wide tiles < 148
+    assert fa.gemm_tiles(3328, 3328, 148) == (256, 13, 13)   # 169 >= 148
+    with pytest.raises(fa.FAError):
+        fa.gemm_tiles(0, 5, 148)

@@ -51,8 +51,10 @@ def test_square_sizes(n):
 
 @pytest.mark.parametrize("M,N,K", [(1, 128, 64), (256, 1, 64), (256, 128, 1), (17, 300, 129),
                                    (513, 130, 70), (1792, 1792, 64), (1793, 1793, 64),
-                                   (2304, 2304, 256), (4096, 256, 4096), (300, 4100, 33)])
+                                   (2304, 2304, 256), (4096, 256, 4096), (300, 4100, 33),
+                                   (3333, 3400, 100), (4096, 4100, 72), (4100, 4096, 1)])
 def test_rectangular_and_wave_edges(M, N, K):
+    """Ragged edges in both tilings (256 x 256 is used from 148 wide tiles up)."""
     a, b = _mats(M, N, K, seed=M + N + K)
     c = _fa().gemm(a.to(DEV), b.to(DEV))
     _fa().check_device_errors()

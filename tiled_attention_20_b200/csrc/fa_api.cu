@@ -488,6 +488,28 @@ int make_tmap_2d(CUtensorMap* m, const void* base, int rows, int cols, int ld, i
   return r == CUDA_SUCCESS ? FA_OK : FA_ERR_LAUNCH;
 }
 
+// Tile width: 256 columns when that still gives every SM at least one tile,
+// else 128 (more, smaller tiles for small problems).
+int gemm_tile_n(int M, int N, int sms) {
+  const long long t256 = static_cast<long long>((M + fa::kGemmBM - 1) / fa::kGemmBM) * ((N + 255) / 256);
+  return t256 >= sms ? 256 : 128;
+}
+
+template <int BN>
+int launch_gemm_t(const CUtensorMap& ta, const CUtensorMap& tb, fa::GemmParams p, int sms,
+                  cudaStream_t st) {
+  p.tiles_n = (p.N + BN - 1) / BN;
+  p.n_tiles = ((p.M + fa::kGemmBM - 1) / fa::kGemmBM) * p.tiles_n;
+  const int ctas = p.n_tiles < sms ? p.n_tiles : sms;
+  auto kern = fa::fa_gemm_kernel<BN>;
+  const int smem = fa::GemmLayout<BN>::kSmemBytes;
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
+    return FA_ERR_LAUNCH;
+  LaunchTrace trace(kKernGemm, st);
+  kern<<<ctas, 256, smem, st>>>(ta, tb, p);
+  return cudaPeekAtLastError() == cudaSuccess ? FA_OK : FA_ERR_LAUNCH;
+}
+
 int launch_gemm_pack(const void* src, int ld_src, void* dst, int ld_dst, int rows, int cols,
                      int sms, cudaStream_t stream) {
   LaunchTrace trace(kKernGemmPack, stream);
@@ -656,11 +678,12 @@ size_t fa_gemm_workspace_size(const void* A, const void* B, int M, int N, int K,
   return gemm_ws_bytes(A, B, M, N, K, lda, ldb);
 }
 
-int fa_gemm_tiles(int M, int N, int* tiles_m, int* tiles_n) {
-  if (!tiles_m || !tiles_n) return FA_ERR_NULL;
-  if (M < 1 || N < 1) return FA_ERR_SHAPE;
+int fa_gemm_tiles(int M, int N, int sms, int* tile_n, int* tiles_m, int* tiles_n) {
+  if (!tile_n || !tiles_m || !tiles_n) return FA_ERR_NULL;
+  if (M < 1 || N < 1 || sms < 1) return FA_ERR_SHAPE;
+  *tile_n = gemm_tile_n(M, N, sms);
   *tiles_m = (M + fa::kGemmBM - 1) / fa::kGemmBM;
-  *tiles_n = (N + fa::kGemmBN - 1) / fa::kGemmBN;
+  *tiles_n = (N + *tile_n - 1) / *tile_n;
   return FA_OK;
 }
 
@@ -709,18 +732,10 @@ int fa_gemm(const void* A, const void* B, void* C, int M, int N, int K, int lda,
   p.N = N;
   p.K = K;
   p.ldc = ldc;
-  p.tiles_n = (N + fa::kGemmBN - 1) / fa::kGemmBN;
-  p.n_tiles = ((M + fa::kGemmBM - 1) / fa::kGemmBM) * p.tiles_n;
   p.k_blocks = (K + fa::kGemmBK - 1) / fa::kGemmBK;
   p.status = info->status;
-  const int ctas = p.n_tiles < info->sms ? p.n_tiles : info->sms;
-  auto kern = fa::fa_gemm_kernel;
-  const int smem = fa::GemmLayout::kSmemBytes;
-  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
-    return FA_ERR_LAUNCH;
-  LaunchTrace trace(kKernGemm, st);
-  kern<<<ctas, 256, smem, st>>>(ta, tb, p);
-  return cudaPeekAtLastError() == cudaSuccess ? FA_OK : FA_ERR_LAUNCH;
+  return gemm_tile_n(M, N, info->sms) == 256 ? launch_gemm_t<256>(ta, tb, p, info->sms, st)
+                                             : launch_gemm_t<128>(ta, tb, p, info->sms, st);
 }
 
 int fa_fwd_fp8(const void* q, const void* k, const void* v, const float* descale_q,

@@ -6,17 +6,20 @@
 // their alignment), and the curve steps down whenever the count of output
 // tiles crosses a multiple of the SM count (wave quantization).
 //
-// B200 design: one persistent CTA per SM walks the 256 x 128 output tiles
-// (the tile shape of that example) in a static round-robin order, so the
-// number of tiles over 148 SMs sets the number of rounds.  Per CTA:
+// B200 design: one persistent CTA per SM walks the 256 x BN output tiles in
+// a static round-robin order, so the number of tiles over 148 SMs sets the
+// number of rounds.  BN = 128 is the tile shape of that example; BN = 256
+// halves the operand traffic per FLOP (A is reused for twice the columns)
+// and is used whenever it still gives every SM a tile.  Per CTA:
 //   warp 0      TMA producer: per 64-wide K block, A as two 128 x 64 boxes
-//               (K-major) and B as two 64 x 64 boxes (row-major B is
-//               MN-major for the tensor core), 128-byte swizzle, 4 stages;
+//               (K-major) and B as BN/64 boxes of 64 x 64 (row-major B is
+//               MN-major for the tensor core), 128-byte swizzle;
 //   warp 1      TMEM allocator and single-thread tcgen05.mma issuer:
-//               M = 128, N = 128, K = 16 per instruction, two M halves;
+//               M = 128, N = BN, K = 16 per instruction, two M halves;
 //   warps 4-7   epilogue: TMEM -> registers -> bf16 -> global memory.
-// TMEM holds two 256-column accumulators (two M halves of 128 columns each)
-// so the epilogue of one tile overlaps the main loop of the next.
+// With BN = 128 TMEM holds two 256-column accumulators, so the epilogue of
+// one tile overlaps the main loop of the next; with BN = 256 the one
+// accumulator fills all 512 columns and the epilogue runs between tiles.
 // Ragged M, N, K edges read zeros from the TMA out-of-bounds fill; the
 // epilogue checks rows and columns.  TMA needs 16-byte aligned row strides:
 // the host packs an operand whose leading dimension is not a multiple of 8
@@ -28,15 +31,17 @@
 namespace fa {
 
 constexpr int kGemmBM = 256;
-constexpr int kGemmBN = 128;
 constexpr int kGemmBK = 64;
-constexpr int kGemmStages = 4;
+constexpr int kGemmMaxStages = 4;
 
+template <int BN>
 struct GemmLayout {
-  static constexpr int kABytes = kGemmBM * kGemmBK * 2;  // two 128 x 64 boxes, 16 KB each
-  static constexpr int kBBytes = kGemmBK * kGemmBN * 2;  // two 64 x 64 boxes, 8 KB each
+  static constexpr int kStages = BN == 128 ? 4 : 3;
+  static constexpr int kAccBufs = BN == 128 ? 2 : 1;       // accumulators in 512 TMEM columns
+  static constexpr int kABytes = kGemmBM * kGemmBK * 2;   // two 128 x 64 boxes, 16 KB each
+  static constexpr int kBBytes = kGemmBK * BN * 2;        // BN/64 boxes of 64 x 64, 8 KB each
   static constexpr int kStageBytes = kABytes + kBBytes;
-  static constexpr int kBar = kGemmStages * kStageBytes;
+  static constexpr int kBar = kStages * kStageBytes;
   static constexpr int kSmemBytes = kBar + 256 + 1024;  // + manual 1024-byte alignment
 };
 
@@ -48,7 +53,7 @@ struct GemmParams {
 };
 
 struct GemmBarriers {
-  uint64_t full[kGemmStages], empty[kGemmStages];
+  uint64_t full[kGemmMaxStages], empty[kGemmMaxStages];
   uint64_t acc_full[2], acc_empty[2];
   uint64_t mma_done;
   uint32_t tmem_base;
@@ -81,11 +86,13 @@ __device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* m, uin
       : "memory");
 }
 
+template <int BN>
 __global__ void __launch_bounds__(256, 1)
     fa_gemm_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_b,
                    const GemmParams p) {
-  using L = GemmLayout;
-  constexpr int S = kGemmStages;
+  using L = GemmLayout<BN>;
+  constexpr int S = L::kStages;
+  constexpr int NB = L::kAccBufs;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
@@ -124,7 +131,7 @@ __global__ void __launch_bounds__(256, 1)
     if (lane_id() == 0) {
       int it = 0;
       for (int tile = blockIdx.x; tile < p.n_tiles; tile += G) {
-        const int m0 = (tile / p.tiles_n) * kGemmBM, n0 = (tile % p.tiles_n) * kGemmBN;
+        const int m0 = (tile / p.tiles_n) * kGemmBM, n0 = (tile % p.tiles_n) * BN;
         for (int kb = 0; kb < p.k_blocks; ++kb, ++it) {
           const int st = it % S;
           if (it >= S && !gemm_wait1(&b->empty[st], ((it / S) - 1) & 1, b, p.status)) goto drain;
@@ -134,8 +141,9 @@ __global__ void __launch_bounds__(256, 1)
           const int k0 = kb * kGemmBK;
           tma_load_2d(sa, &tm_a, &b->full[st], k0, m0);
           tma_load_2d(sa + 16384, &tm_a, &b->full[st], k0, m0 + 128);
-          tma_load_2d(sb, &tm_b, &b->full[st], n0, k0);
-          tma_load_2d(sb + 8192, &tm_b, &b->full[st], n0 + 64, k0);
+#pragma unroll
+          for (int j = 0; j < BN / 64; ++j)
+            tma_load_2d(sb + 8192 * j, &tm_b, &b->full[st], n0 + 64 * j, k0);
         }
       }
     drain:
@@ -149,14 +157,14 @@ __global__ void __launch_bounds__(256, 1)
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
     if (lane_id() == 0) {
-      constexpr uint32_t idesc = idesc_bf16_f32(128, 128, false, true);
+      constexpr uint32_t idesc = idesc_bf16_f32(128, BN, false, true);
       const uint32_t sbase = smem_u32(smem);
       int it = 0, tc = 0;
       for (int tile = blockIdx.x; tile < p.n_tiles; tile += G, ++tc) {
-        const int buf = tc & 1;
-        if (tc >= 2 && !gemm_wait1(&b->acc_empty[buf], ((tc >> 1) - 1) & 1, b, p.status)) break;
+        const int buf = tc % NB, use = tc / NB;
+        if (use >= 1 && !gemm_wait1(&b->acc_empty[buf], (use - 1) & 1, b, p.status)) break;
         tc_fence_after();
-        const uint32_t acc = tmem + buf * 256;
+        const uint32_t acc = tmem + buf * 2 * BN;
         bool ok = true;
         for (int kb = 0; kb < p.k_blocks; ++kb, ++it) {
           const int st = it % S;
@@ -171,7 +179,7 @@ __global__ void __launch_bounds__(256, 1)
           for (int h = 0; h < 2; ++h)
 #pragma unroll
             for (int kk = 0; kk < 4; ++kk)
-              mma_ss(acc + h * 128, sdesc_sw128(sa + h * 16384 + kk * 32, 16, 1024),
+              mma_ss(acc + h * BN, sdesc_sw128(sa + h * 16384 + kk * 32, 16, 1024),
                      sdesc_sw128(sb + kk * 2048, 8192, 1024), idesc, (kb > 0 || kk > 0) ? 1u : 0u);
           mma_commit(&b->empty[st]);
         }
@@ -189,17 +197,17 @@ __global__ void __launch_bounds__(256, 1)
     const bool vec_ok = (p.ldc % 8) == 0 && (reinterpret_cast<uintptr_t>(p.c) & 15) == 0;
     int tc = 0;
     for (int tile = blockIdx.x; tile < p.n_tiles; tile += G, ++tc) {
-      const int buf = tc & 1;
-      if (!gemm_wait_warp(&b->acc_full[buf], (tc >> 1) & 1, b, p.status)) break;
+      const int buf = tc % NB;
+      if (!gemm_wait_warp(&b->acc_full[buf], (tc / NB) & 1, b, p.status)) break;
       tc_fence_after();
-      const int m0 = (tile / p.tiles_n) * kGemmBM, n0 = (tile % p.tiles_n) * kGemmBN;
+      const int m0 = (tile / p.tiles_n) * kGemmBM, n0 = (tile % p.tiles_n) * BN;
 #pragma unroll 1
       for (int h = 0; h < 2; ++h) {
         const int row = m0 + 128 * h + t;
 #pragma unroll 1
-        for (int c0 = 0; c0 < kGemmBN; c0 += 32) {
+        for (int c0 = 0; c0 < BN; c0 += 32) {
           uint32_t r[32];
-          tmem_ld_x32(tmem + lane_base + buf * 256 + h * 128 + c0, r);
+          tmem_ld_x32(tmem + lane_base + buf * 2 * BN + h * BN + c0, r);
           uint16_t* dst = p.c + static_cast<size_t>(row) * p.ldc + n0 + c0;
           const int ncols = row < p.M ? min(32, p.N - (n0 + c0)) : 0;
           if (vec_ok && ncols == 32) {

@@ -84,7 +84,8 @@ def load(path: str = LIB_PATH):
         lib.fa_gemm.restype = _i
         lib.fa_gemm_workspace_size.argtypes = [_vp, _vp, _i, _i, _i, _i, _i]
         lib.fa_gemm_workspace_size.restype = _sz
-        lib.fa_gemm_tiles.argtypes = [_i, _i, ctypes.POINTER(_i), ctypes.POINTER(_i)]
+        lib.fa_gemm_tiles.argtypes = [_i, _i, _i, ctypes.POINTER(_i), ctypes.POINTER(_i),
+                                      ctypes.POINTER(_i)]
         lib.fa_gemm_tiles.restype = _i
         lib.fa_fwd_fp8.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _f,
                                    _i, _vp]
@@ -321,11 +322,12 @@ def decode(q, k_cache, v_cache, cache_lens=None, scale=None, causal=False, nk=No
     return out, lse
 
 
-def gemm_tiles(M, N):
-    """(tiles_m, tiles_n) of fa_gemm's 256 x 128 output tiles."""
-    tm, tn = _i(0), _i(0)
-    _check(load().fa_gemm_tiles(M, N, ctypes.byref(tm), ctypes.byref(tn)), "fa_gemm_tiles")
-    return tm.value, tn.value
+def gemm_tiles(M, N, sms=148):
+    """(tile_n, tiles_m, tiles_n): fa_gemm's tiles are 256 x tile_n."""
+    bn, tm, tn = _i(0), _i(0), _i(0)
+    _check(load().fa_gemm_tiles(M, N, sms, ctypes.byref(bn), ctypes.byref(tm), ctypes.byref(tn)),
+           "fa_gemm_tiles")
+    return bn.value, tm.value, tn.value
 
 
 def _ld(t):
