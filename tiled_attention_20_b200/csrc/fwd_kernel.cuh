@@ -90,6 +90,7 @@ struct FwdBarriers {
   uint64_t q_full, q_empty;
   uint64_t k_full[4], k_empty[4], v_full[4], v_empty[4];
   uint64_t s_full[2], p_full[2], o_full[2];
+  uint64_t p_half[2];  // bf16: the first 64 keys of P are in TMEM
   uint64_t mma_done;
   uint32_t tmem_base;
   int abort_flag;
@@ -219,7 +220,8 @@ __device__ __forceinline__ void issue_s(uint32_t tmem_s, uint32_t q_smem, uint32
 // O += P V: A = P from TMEM (8 columns per K-step in both types: 16 bf16 or
 // 32 E4M3 keys), B = V MN-major (a K-step covers 16 or 32 key rows of 128
 // bytes; bf16 rows of D = 128 span two 64-column boxes 16 KB apart).
-template <int D, bool FP8>
+// HALF = 0 / 1 issues only the K-steps of keys 0-63 / 64-127 (bf16).
+template <int D, bool FP8, int HALF = -1>
 __device__ __forceinline__ void issue_pv(uint32_t tmem_o, uint32_t tmem_p, uint32_t v_smem,
                                          bool accumulate) {
   if constexpr (FP8) {
@@ -231,7 +233,7 @@ __device__ __forceinline__ void issue_pv(uint32_t tmem_o, uint32_t tmem_p, uint3
   } else {
     constexpr uint32_t idesc = idesc_bf16_f32(128, D, false, true);
 #pragma unroll
-    for (int kk = 0; kk < 8; ++kk)
+    for (int kk = (HALF == 1 ? 4 : 0); kk < (HALF == 0 ? 4 : 8); ++kk)
       mma_ts(tmem_o, tmem_p + kk * 8, sdesc_sw128(v_smem + kk * 2048, 16384, 1024), idesc,
              (accumulate || kk > 0) ? 1u : 0u);
   }
@@ -240,6 +242,23 @@ __device__ __forceinline__ void issue_pv(uint32_t tmem_o, uint32_t tmem_p, uint3
 template <int D, bool CAUSAL, bool FP8>
 __device__ void fwd_mma(const FwdParams& p, uint8_t* smem, FwdBarriers* b, uint32_t tmem) {
   using L = FwdLayout<D, FP8>;
+  // O_i += P_i V for Q tile i.  bf16: the keys 0-63 half is issued as soon
+  // as the softmax has stored it, the rest when the whole P is in TMEM.
+  auto pv = [&](int i, int& pcount, uint32_t to, uint32_t ts, uint32_t v_smem, bool acc) -> bool {
+    if constexpr (!FP8) {
+      if (!wait1(&b->p_half[i], pcount & 1, b, p.status)) return false;
+      tc_fence_after();
+      issue_pv<D, FP8, 0>(to, ts, v_smem, acc);
+    }
+    if (!wait1(&b->p_full[i], pcount & 1, b, p.status)) return false;
+    ++pcount;
+    tc_fence_after();
+    if constexpr (!FP8)
+      issue_pv<D, FP8, 1>(to, ts, v_smem, true);
+    else
+      issue_pv<D, FP8>(to, ts, v_smem, acc);
+    return true;
+  };
   constexpr int S = L::kStages;
   const uint32_t sb = smem_u32(smem);
   const uint32_t tS[2] = {tmem + 0, tmem + 128};
@@ -267,10 +286,7 @@ __device__ void fwd_mma(const FwdParams& p, uint8_t* smem, FwdBarriers* b, uint3
         tc_fence_after();
       }
       if (j >= 1 && j - 1 < nk0) {
-        if (!wait1(&b->p_full[0], pc[0] & 1, b, p.status)) return;
-        ++pc[0];
-        tc_fence_after();
-        issue_pv<D, FP8>(tO[0], tS[0], v_smem, j - 1 > 0);
+        if (!pv(0, pc[0], tO[0], tS[0], v_smem, j - 1 > 0)) return;
         if (j - 1 == nk0 - 1) mma_commit(&b->o_full[0]);
       }
       if (j < nk0) {
@@ -278,10 +294,7 @@ __device__ void fwd_mma(const FwdParams& p, uint8_t* smem, FwdBarriers* b, uint3
         mma_commit(&b->s_full[0]);
       }
       if (j >= 1 && j - 1 < nk1) {
-        if (!wait1(&b->p_full[1], pc[1] & 1, b, p.status)) return;
-        ++pc[1];
-        tc_fence_after();
-        issue_pv<D, FP8>(tO[1], tS[1], v_smem, j - 1 > 0);
+        if (!pv(1, pc[1], tO[1], tS[1], v_smem, j - 1 > 0)) return;
         if (j - 1 == nk1 - 1) mma_commit(&b->o_full[1]);
       }
       if (j >= 1) {
@@ -302,17 +315,11 @@ __device__ void fwd_mma(const FwdParams& p, uint8_t* smem, FwdBarriers* b, uint3
     if (!wait1(&b->v_full[vs], (vc / S) & 1, b, p.status)) return;
     tc_fence_after();
     if (nk - 1 < nk0) {
-      if (!wait1(&b->p_full[0], pc[0] & 1, b, p.status)) return;
-      ++pc[0];
-      tc_fence_after();
-      issue_pv<D, FP8>(tO[0], tS[0], v_smem, nk - 1 > 0);
+      if (!pv(0, pc[0], tO[0], tS[0], v_smem, nk - 1 > 0)) return;
       mma_commit(&b->o_full[0]);
     }
     if (nk - 1 < nk1) {
-      if (!wait1(&b->p_full[1], pc[1] & 1, b, p.status)) return;
-      ++pc[1];
-      tc_fence_after();
-      issue_pv<D, FP8>(tO[1], tS[1], v_smem, nk - 1 > 0);
+      if (!pv(1, pc[1], tO[1], tS[1], v_smem, nk - 1 > 0)) return;
       mma_commit(&b->o_full[1]);
     }
     mma_commit(&b->v_empty[vs]);
@@ -443,7 +450,9 @@ __device__ void fwd_softmax(const FwdParams& p, FwdBarriers* b, uint32_t tmem, i
       float2 rs[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f),
                       make_float2(0.f, 0.f)};
       // P in two halves of 64 keys; each half is stored as soon as it is
-      // packed (S is already in registers, so overwriting it is safe).  On
+      // packed (S is already in registers, so overwriting it is safe), and
+      // for bf16 the first half is published at once, so the P V MMA of
+      // keys 0-63 overlaps the exponentials of keys 64-127.  On
       // unmasked tiles 3 of every 8 pairs take the polynomial exp2 on the
       // FMA pipe and the rest the MUFU unit; masked tiles (which hold -inf)
       // use the MUFU unit throughout so masked probabilities are exactly 0.
@@ -465,6 +474,12 @@ __device__ void fwd_softmax(const FwdParams& p, FwdBarriers* b, uint32_t tmem, i
             pk[q2] = pack_bf16x2(pp.x, pp.y);
           }
           tmem_st_x32(tS + 32 * h, pk);
+          if (h == 0) {  // keys 0-63 of P are ready: the MMA may start on them
+            tmem_st_wait();
+            tc_fence_before();
+            __syncwarp();
+            if (lane_id() == 0) mbar_arrive(&b->p_half[wg]);
+          }
         }
       } else {
 #pragma unroll
@@ -480,6 +495,12 @@ __device__ void fwd_softmax(const FwdParams& p, FwdBarriers* b, uint32_t tmem, i
             pk[q2] = pack_bf16x2(pp.x, pp.y);
           }
           tmem_st_x32(tS + 32 * h, pk);
+          if (h == 0) {  // keys 0-63 of P are ready: the MMA may start on them
+            tmem_st_wait();
+            tc_fence_before();
+            __syncwarp();
+            if (lane_id() == 0) mbar_arrive(&b->p_half[wg]);
+          }
         }
       }
       const float2 rsum = add2(add2(rs[0], rs[1]), add2(rs[2], rs[3]));
@@ -540,6 +561,7 @@ __global__ void __launch_bounds__(384, 1)
     for (int i = 0; i < 2; ++i) {
       mbar_init(&b->s_full[i], 1);
       mbar_init(&b->p_full[i], 4);
+      mbar_init(&b->p_half[i], 4);
       mbar_init(&b->o_full[i], 1);
     }
     mbar_init(&b->mma_done, 1);
