@@ -157,6 +157,15 @@ const char *fa_strerror(int status);
  * FA_ERR_LAUNCH (a CUDA error is pending on the device). */
 int fa_check_device_errors(fa_stream_t stream);
 
+/* Failure-detection self-test (no counterpart on the pages: a test hook).
+ * Enqueues a one-thread kernel whose wait on an mbarrier can never complete;
+ * the wait gives up after limit_ms (1..2000) milliseconds exactly as the
+ * library's kernels' bounded waits do, latches the timeout bit in the status
+ * word and returns, so the next fa_check_device_errors() reports
+ * FA_ERR_TIMEOUT and the CUDA context stays usable.  Nothing hangs or
+ * faults.  Returns FA_OK once enqueued, FA_ERR_ARG for a limit out of range. */
+int fa_selftest_wait_timeout(int limit_ms, fa_stream_t stream);
+
 /* Number of persistent CTAs fa_fwd / fa_bwd launch for a problem on the
  * current device (pass = 0 forward, 1 backward), and the number of work
  * units they share; for the harness and its wave-quantization checks.

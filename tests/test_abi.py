@@ -154,3 +154,8 @@ def test_gemm_tiles(lib):
     assert fa.gemm_tiles(3328, 3328, 148) == (256, 13, 13)   # 169 >= 148
     with pytest.raises(fa.FAError):
         fa.gemm_tiles(0, 5, 148)
+
+
+def test_selftest_limit_validation(lib):
+    assert lib.fa_selftest_wait_timeout(0, None) == -10
+    assert lib.fa_selftest_wait_timeout(2001, None) == -10

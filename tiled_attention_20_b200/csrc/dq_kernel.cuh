@@ -78,11 +78,25 @@ struct DqUnit {
   int bh, q0, nk;  // head, first query row, key tiles visited
 };
 
+// Work unit w -> (head, Q tile), ordered as the forward's units: longest
+// first across heads when causal, heads in groups of kDqHeadGroup (shared K
+// and V in L2) otherwise.
+constexpr int kDqHeadGroup = 8;
+
 template <bool CAUSAL>
 __device__ __forceinline__ DqUnit dq_decode(const DqParams& p, int w) {
   DqUnit u;
-  const int idx = w / p.BH;
-  u.bh = w - idx * p.BH;
+  int idx;
+  if (CAUSAL) {
+    idx = w / p.BH;
+    u.bh = w - idx * p.BH;
+  } else {
+    const int g = w / (kDqHeadGroup * p.nqt), g0 = g * kDqHeadGroup;
+    const int gs = min(kDqHeadGroup, p.BH - g0);
+    const int r = w - g * kDqHeadGroup * p.nqt;
+    idx = r / gs;
+    u.bh = g0 + (r - idx * gs);
+  }
   const int qt = CAUSAL ? (p.nqt - 1 - idx) : idx;  // causal: longest first
   u.q0 = qt * 128;
   const int nkv = (p.N + 127) / 128;

@@ -24,6 +24,18 @@ namespace {
 // Per-device status word the kernels OR error bits into.
 __device__ int g_fa_status;
 
+// Failure-detection self-test: one thread waits, with the given bound, on an
+// mbarrier that nothing will ever arrive on.  The bounded wait gives up,
+// latches the timeout bit and the kernel returns normally.
+__global__ void fa_selftest_timeout_kernel(int* status, unsigned long long limit_ns) {
+  __shared__ uint64_t bar;
+  if (threadIdx.x == 0) {
+    fa::mbar_init(&bar, 1);
+    fa::fence_barrier_init();
+    fa::mbar_wait(&bar, 0, status, limit_ns);  // phase 0 never completes
+  }
+}
+
 constexpr int kMaxDevices = 64;
 
 struct DeviceInfo {
@@ -818,6 +830,16 @@ int fa_bwd(const void* q, const void* k, const void* v, const void* o, const voi
   if ((s = device_info(&info)) != FA_OK) return s;
   return launch_bwd(q, k, v, o, dO, lse, dq, dk, dv, B, H, N, d, scale, causal != 0, workspace,
                     grad_dtype, info->sms, info->status, reinterpret_cast<cudaStream_t>(stream));
+}
+
+int fa_selftest_wait_timeout(int limit_ms, fa_stream_t stream) {
+  if (limit_ms < 1 || limit_ms > 2000) return FA_ERR_ARG;
+  DeviceInfo* info = nullptr;
+  int s = device_info(&info);
+  if (s != FA_OK) return s;
+  fa_selftest_timeout_kernel<<<1, 32, 0, reinterpret_cast<cudaStream_t>(stream)>>>(
+      info->status, static_cast<unsigned long long>(limit_ms) * 1000000ull);
+  return cudaPeekAtLastError() == cudaSuccess ? FA_OK : FA_ERR_LAUNCH;
 }
 
 int fa_check_device_errors(fa_stream_t stream) {

@@ -100,11 +100,27 @@ struct FwdUnit {
   int bh, q0, nk0, nk1;
 };
 
+// Work unit w -> (head, Q tile pair).  Causal: tile-pair index major, head
+// minor, so units come longest first across all heads (load balance).
+// Non-causal (all units equal): heads in groups of kUnitHeadGroup, tile
+// pair major within a group, so the CTAs running at one time share a few
+// heads' K and V in L2 instead of streaming every head's.
+constexpr int kUnitHeadGroup = 8;
+
 template <bool CAUSAL>
 __device__ __forceinline__ FwdUnit fwd_decode(const FwdParams& p, int w) {
   FwdUnit u;
-  const int idx = w / p.BH;
-  u.bh = w - idx * p.BH;
+  int idx;
+  if (CAUSAL) {
+    idx = w / p.BH;
+    u.bh = w - idx * p.BH;
+  } else {
+    const int g = w / (kUnitHeadGroup * p.n_qt2), g0 = g * kUnitHeadGroup;
+    const int gs = min(kUnitHeadGroup, p.BH - g0);
+    const int r = w - g * kUnitHeadGroup * p.n_qt2;  // every earlier group is full
+    idx = r / gs;
+    u.bh = g0 + (r - idx * gs);
+  }
   const int qt2 = CAUSAL ? (p.n_qt2 - 1 - idx) : idx;
   u.q0 = qt2 * 256;
   const int nkv = (p.N + 127) / 128;

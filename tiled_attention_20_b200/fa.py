@@ -29,7 +29,7 @@ EXPORTED = ["fa_fwd", "fa_bwd", "fa_bwd_workspace_size", "fa_strerror",
             "fa_check_device_errors", "fa_launch_shape", "fa_trace_start", "fa_trace_stop",
             "fa_trace_kernel_name", "fa_bwd_noalloc", "fa_bwd_deterministic",
             "fa_decode", "fa_decode_workspace_size", "fa_decode_plan", "fa_fwd_fp8",
-            "fa_gemm", "fa_gemm_workspace_size", "fa_gemm_tiles"]
+            "fa_gemm", "fa_gemm_workspace_size", "fa_gemm_tiles", "fa_selftest_wait_timeout"]
 NOALLOC_MAX_SCRATCH = 32 << 20  # FA_BWD_NOALLOC_MAX_SCRATCH
 KERNEL_IDS = {0: "fa_fwd_kernel", 1: "fa_bwd_prep", 2: "fa_bwd_kernel", 3: "fa_bwd_dq_convert",
               4: "fa_dq_kernel", 5: "fa_decode_kernel", 6: "fa_gemm_kernel", 7: "fa_gemm_pack"}
@@ -80,6 +80,8 @@ def load(path: str = LIB_PATH):
         lib.fa_bwd_noalloc.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp,
                                        _i, _i, _i, _i, _f, _i, _i, _vp]
         lib.fa_bwd_noalloc.restype = _i
+        lib.fa_selftest_wait_timeout.argtypes = [_i, _vp]
+        lib.fa_selftest_wait_timeout.restype = _i
         lib.fa_gemm.argtypes = [_vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _vp, _sz, _vp]
         lib.fa_gemm.restype = _i
         lib.fa_gemm_workspace_size.argtypes = [_vp, _vp, _i, _i, _i, _i, _i]
@@ -358,3 +360,12 @@ def gemm(a, b, out=None, workspace=None):
                             workspace.data_ptr(), workspace.numel(), _stream(a.device))
     _check(st, "fa_gemm")
     return out
+
+
+def selftest_wait_timeout(limit_ms=50, device=None):
+    """Enqueue the failure-detection self-test (a bounded wait that must time
+    out after limit_ms); the next check_device_errors() raises FA_ERR_TIMEOUT."""
+    device = torch.cuda.current_device() if device is None else device
+    with torch.cuda.device(device):
+        _check(load().fa_selftest_wait_timeout(int(limit_ms), _stream(device)),
+               "fa_selftest_wait_timeout")
