@@ -502,7 +502,9 @@ def run_gemm_sweep(args, rank, world, local_rank, dist):
     clocks = sampler.stop()
     fa.check_device_errors(dev)
     top = next((r for r in sweep if r["N"] == 8192), max(sweep, key=lambda r: r["N"]))
-    value = top["tflops"] * world
+    # whole-job rate: every rank ran the same point; the slowest rank sets the time
+    top_ms = ranks.max_over_ranks(top["ms"], dist, dev)
+    value = 2.0 * top["N"] ** 3 * world / top_ms / 1e9
     roof = {"bound": "tensor", "achieved": top["tflops"], "peak": peaks["bf16_tflops"],
             "unit": "TFLOP/s", "frac": top["tflops"] / peaks["bf16_tflops"],
             "traffic": profiled_traffic(f"fa_gemm_kernel:{top['N']}"),

@@ -4,8 +4,9 @@ bench.py times (fa.fwd + fa.bwd with a library-sized workspace).
 The fp64 oracle cannot do every head of the large workloads in test time, so
 it checks whole heads sampled from each problem (all rows and gradients of
 those heads); properties that hold at any size are checked on every head:
-causal row 0 equals V_0 bit for bit and its lse equals scale*q_0.k_0, and the
-outputs are finite."""
+causal row 0 equals V_0 bit for bit and its lse equals scale*q_0.k_0, the
+gradient sum rules (sum_j dK_j = 0, sum_j dV_j = sum_i dO_i) hold within the
+kernel's rounding bounds, and the outputs are finite."""
 import math
 
 import numpy as np
@@ -52,7 +53,7 @@ def _check_heads(w, cpu_in, gpu_out, heads, scaled=False):
 
 
 def _check_all_heads_properties(w, cpu_in, gpu_out):
-    q, k, v, _ = cpu_in
+    q, k, v, dO = cpu_in
     o, lse, dq, dk, dv = gpu_out
     for t in (o, lse, dq, dk, dv):
         assert torch.isfinite(t.float()).all()
@@ -60,6 +61,23 @@ def _check_all_heads_properties(w, cpu_in, gpu_out):
         assert torch.equal(o[:, :, 0], v[:, :, 0])
         s00 = (q[:, :, 0].double() * k[:, :, 0].double()).sum(-1) / math.sqrt(w.d)
         assert np.abs(np64(lse[:, :, 0]) - s00.numpy()).max() <= 1e-3 * max(1.0, float(s00.abs().max()))
+    # Gradient sum rules on every head: key-shift invariance gives
+    # sum_j dK_j = 0, rows of P summing to one give sum_j dV_j = sum_i dO_i.
+    # Bounds from the kernel's rounding model, doubled: bf16 operands P and dS
+    # (relative 2^-9), D formed from the bf16 O, and the bf16 rounding of each
+    # output element (another 2^-9 relative).
+    u = 2.0 ** -9
+    scale = 1 / math.sqrt(w.d)
+    for bi in range(w.B):  # one batch entry at a time keeps host memory small
+        dk64, dv64, dO64, q64, o64 = (np64(t[bi]) for t in (dk, dv, dO, q, o))
+        dd = np.abs(dO64 * o64).sum(axis=2, keepdims=True)
+        bound_k = 2 * (2 * u * np.abs(dk64).sum(axis=1)
+                       + scale * u * (dd * np.abs(q64)).sum(axis=1)) + 1e-6
+        err_k = np.abs(dk64.sum(axis=1))
+        assert (err_k <= bound_k).all(), f"sum dK: {err_k.max():.3e} (batch {bi})"
+        bound_v = 2 * u * (np.abs(dO64).sum(axis=1) + np.abs(dv64).sum(axis=1)) + 1e-6
+        assert (np.abs(dv64.sum(axis=1) - dO64.sum(axis=1)) <= bound_v).all(), \
+            f"sum dV != sum dO (batch {bi})"
 
 
 def test_gpt_causal_workload():
