@@ -13,7 +13,9 @@
  * probabilities instead of storing them ("CS336 Lecture 5 · GPUs, TPUs"
  * notes, section "FlashAttention 解析", item ② on recomputation).
  *
- * Conventions shared by every entry point:
+ * Conventions shared by the attention entry points (fa_fwd, fa_fwd_fp8,
+ * fa_bwd, fa_bwd_deterministic, fa_bwd_noalloc; fa_decode and fa_gemm state
+ * their own shapes):
  *   - Tensors Q, K, V, O, dO, dQ, dK, dV are dense row-major [B, H, N, d]
  *     (d contiguous, then N, then H, then B), bf16 unless stated.  lse and
  *     the backward's D are [B, H, N] fp32.  Queries and keys share length N.
@@ -29,11 +31,12 @@
  *     crosses the ABI.
  *   - Calls are thread-safe.  Two calls that run concurrently on the GPU must
  *     not share output or workspace buffers.
- *   - Results are deterministic for the forward, dK and dV.  The backward
- *     sums the per-block dQ contributions with fp32 reduce-add copies whose
- *     order varies, so dQ may differ in the last bits between runs (the
- *     pages note that tiled attention is not bit-identical to the untiled
- *     computation, §8.4 of the first page).
+ *   - Results are deterministic for the forward, dK and dV.  fa_bwd sums
+ *     the per-block dQ contributions with fp32 reduce-add copies whose order
+ *     varies, so its dQ may differ in the last bits between runs (the pages
+ *     note that tiled attention is not bit-identical to the untiled
+ *     computation, §8.4 of the first page); fa_bwd_deterministic gives a
+ *     run-to-run identical dQ at some cost in speed.
  */
 #ifndef FA_H_
 #define FA_H_
