@@ -139,6 +139,64 @@ def profiled_traffic(kernel: str):
     return None
 
 
+# ---------------------------------------------------------------- end to end
+def pipelined_e2e(dev, host_in, dev_in, dev_out, host_out, run, steps, dist=None):
+    """Per-step milliseconds of host -> device -> host steps through the
+    public API.  Two device buffer sets alternate: step i uploads its inputs
+    (pinned host memory) into set i % 2 on one copy stream, its kernels run on
+    the compute stream once that upload is done, and its results go back to
+    pinned host memory on a second copy stream, so the upload of step i+1 and
+    the download of step i-1 overlap the kernels of step i (the two copy
+    directions use separate copy engines).  Events keep each set's reuse in
+    order.  Every step moves its full inputs in and its full results out.
+      host_in / host_out: lists of pinned host tensors;
+      dev_in / dev_out:   two lists (one per set) of matching device tensors;
+      run(k):             enqueues the step's library calls on set k."""
+    comp = torch.cuda.Stream(dev)
+    up = torch.cuda.Stream(dev)
+    down = torch.cuda.Stream(dev)
+    ev = lambda: torch.cuda.Event(enable_timing=False)
+    up_done = [ev(), ev()]
+    comp_done = [ev(), ev()]
+    down_done = [ev(), ev()]
+    used = [False, False]
+
+    def one(i):
+        k = i % 2
+        with torch.cuda.stream(up):
+            if used[k]:
+                up.wait_event(comp_done[k])  # set k's previous kernels have read their inputs
+            for h, d in zip(host_in, dev_in[k]):
+                d.copy_(h, non_blocking=True)
+            up_done[k].record(up)
+        with torch.cuda.stream(comp):
+            comp.wait_event(up_done[k])
+            if used[k]:
+                comp.wait_event(down_done[k])  # set k's previous results are on the host
+            run(k)
+            comp_done[k].record(comp)
+        with torch.cuda.stream(down):
+            down.wait_event(comp_done[k])
+            for d, h in zip(dev_out[k], host_out):
+                h.copy_(d, non_blocking=True)
+            down_done[k].record(down)
+        used[k] = True
+
+    one(0)
+    one(1)
+    torch.cuda.synchronize(dev)
+    if dist is not None and dist.is_initialized():
+        dist.barrier()
+    t0 = torch.cuda.Event(enable_timing=True)
+    t1 = torch.cuda.Event(enable_timing=True)
+    t0.record(up)
+    for i in range(steps):
+        one(i)
+    t1.record(down)
+    torch.cuda.synchronize(dev)
+    return t0.elapsed_time(t1) / steps
+
+
 # ---------------------------------------------------------------- clocks
 class ClockSampler:
     """nvidia-smi samples of SM clock and throttle reasons every 200 ms."""
@@ -344,40 +402,28 @@ def run_ours(args, rank, world, local_rank, dist):
     # end to end through the public API with host buffers
     e2e = None
     if not args.no_e2e:
-        pin = lambda t: t.pin_memory()
-        hq, hk, hv, hdO = (pin(t) for t in (q_h, k_h, v_h, dO_h))
-        ho = torch.empty(q_h.shape, dtype=torch.bfloat16).pin_memory()
-        hlse = torch.empty((w.B, w.H, w.N), dtype=torch.float32).pin_memory()
-        hdq, hdk, hdv = (torch.empty(q_h.shape, dtype=torch.bfloat16).pin_memory() for _ in range(3))
+        host_in = [t.pin_memory() for t in (q_h, k_h, v_h, dO_h)]
+        host_out = [torch.empty(t.shape, dtype=t.dtype).pin_memory() for t in (o, lse, dq, dk, dv)]
+        dev_in = [[q, k, v, dO], [torch.empty_like(t) for t in (q, k, v, dO)]]
+        dev_out = [[o, lse, dq, dk, dv], [torch.empty_like(t) for t in (o, lse, dq, dk, dv)]]
 
-        def e2e_step():
-            q.copy_(hq, non_blocking=True)
-            k.copy_(hk, non_blocking=True)
-            v.copy_(hv, non_blocking=True)
-            dO.copy_(hdO, non_blocking=True)
-            step()
-            ho.copy_(o, non_blocking=True)
-            hlse.copy_(lse, non_blocking=True)
-            hdq.copy_(dq, non_blocking=True)
-            hdk.copy_(dk, non_blocking=True)
-            hdv.copy_(dv, non_blocking=True)
+        def run(kset):
+            qq, kk, vv, dd = dev_in[kset]
+            oo, ll, gq, gk, gv = dev_out[kset]
+            fa.fwd(qq, kk, vv, causal=w.causal, out=oo, lse=ll)
+            fa.bwd(qq, kk, vv, oo, dd, ll, causal=w.causal, workspace=ws, dq=gq, dk=gk, dv=gv,
+                   deterministic=args.deterministic)
 
-        e2e_step()
-        torch.cuda.synchronize(dev)
-        if world > 1:
-            dist.barrier()
         n_e2e = max(1, args.e2e_steps)
-        e0.record(stream)
-        for _ in range(n_e2e):
-            e2e_step()
-        e1.record(stream)
-        torch.cuda.synchronize(dev)
-        ms_e2e = ranks.max_over_ranks(e0.elapsed_time(e1) / n_e2e, dist, dev)
-        nb = lambda *ts: sum(t.numel() * t.element_size() for t in ts)
+        ms_e2e = ranks.max_over_ranks(
+            pipelined_e2e(dev, host_in, dev_in, dev_out, host_out, run, n_e2e, dist), dist, dev)
+        fa.check_device_errors(dev)
+        nb = lambda ts: sum(t.numel() * t.element_size() for t in ts)
         e2e = {"value": ranks.weak_scaling_rate(flops, world, ms_e2e) / 1e12, "unit": UNIT,
-               "h2d_bytes_per_step": nb(hq, hk, hv, hdO),
-               "d2h_bytes_per_step": nb(ho, hlse, hdq, hdk, hdv), "steps": n_e2e,
-               "ms_per_step": ms_e2e, "api": "tiled_attention_20_b200.fa.fwd/bwd (C ABI)"}
+               "h2d_bytes_per_step": nb(host_in), "d2h_bytes_per_step": nb(host_out),
+               "steps": n_e2e, "ms_per_step": ms_e2e,
+               "pipeline": "two buffer sets; uploads and downloads overlap the kernels",
+               "api": "tiled_attention_20_b200.fa.fwd/bwd (C ABI)"}
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -517,30 +563,21 @@ def run_gemm_sweep(args, rank, world, local_rank, dist):
         ha = torch.randn((n, n), generator=torch.Generator().manual_seed(1)).to(torch.bfloat16).pin_memory()
         hb = torch.randn((n, n), generator=torch.Generator().manual_seed(2)).to(torch.bfloat16).pin_memory()
         hc = torch.empty((n, n), dtype=torch.bfloat16).pin_memory()
-        a = torch.empty_like(ha, device=dev)
-        b = torch.empty_like(hb, device=dev)
-        c = torch.empty((n, n), dtype=torch.bfloat16, device=dev)
+        dev_in = [[torch.empty_like(ha, device=dev), torch.empty_like(hb, device=dev)]
+                  for _ in range(2)]
+        dev_out = [[torch.empty((n, n), dtype=torch.bfloat16, device=dev)] for _ in range(2)]
 
-        def e2e_step():
-            a.copy_(ha, non_blocking=True)
-            b.copy_(hb, non_blocking=True)
-            fa.gemm(a, b, out=c, workspace=ws)
-            hc.copy_(c, non_blocking=True)
+        def run(kset):
+            fa.gemm(dev_in[kset][0], dev_in[kset][1], out=dev_out[kset][0], workspace=ws)
 
-        e2e_step()
-        torch.cuda.synchronize(dev)
-        e0 = torch.cuda.Event(enable_timing=True)
-        e1 = torch.cuda.Event(enable_timing=True)
         k = max(1, args.e2e_steps)
-        e0.record(stream)
-        for _ in range(k):
-            e2e_step()
-        e1.record(stream)
-        torch.cuda.synchronize(dev)
-        ms_e2e = e0.elapsed_time(e1) / k
+        ms_e2e = ranks.max_over_ranks(
+            pipelined_e2e(dev, [ha, hb], dev_in, dev_out, [hc], run, k, dist), dist, dev)
         e2e = {"value": 2.0 * n ** 3 / ms_e2e / 1e9 * world, "unit": UNIT,
                "h2d_bytes_per_step": 2 * n * n * 2, "d2h_bytes_per_step": n * n * 2,
-               "steps": k, "ms_per_step": ms_e2e, "api": "tiled_attention_20_b200.fa.gemm (C ABI)"}
+               "steps": k, "ms_per_step": ms_e2e,
+               "pipeline": "two buffer sets; uploads and downloads overlap the kernels",
+               "api": "tiled_attention_20_b200.fa.gemm (C ABI)"}
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -645,30 +682,25 @@ def run_fp8(args, rank, world, local_rank, dist):
 
     e2e = None
     if not args.no_e2e:
-        hin = [t.pin_memory() for t in host[:3]]
-        ho = torch.empty(o.shape, dtype=torch.bfloat16).pin_memory()
-        hlse = torch.empty(lse.shape, dtype=torch.float32).pin_memory()
+        host_in = [t.pin_memory() for t in host[:3]]
+        host_out = [torch.empty(t.shape, dtype=t.dtype).pin_memory() for t in (o, lse)]
+        dev_in = [[q8, k8, v8], [torch.empty_like(t) for t in (q8, k8, v8)]]
+        dev_out = [[o, lse], [torch.empty_like(t) for t in (o, lse)]]
 
-        def e2e_step():
-            for dst, src in zip((q8, k8, v8), hin):
-                dst.copy_(src, non_blocking=True)
-            step()
-            ho.copy_(o, non_blocking=True)
-            hlse.copy_(lse, non_blocking=True)
+        def run(kset):
+            qq, kk, vv = dev_in[kset]
+            fa.fwd_fp8(qq, kk, vv, fq, fk, fv, causal=w.causal, out=dev_out[kset][0],
+                       lse=dev_out[kset][1])
 
-        e2e_step()
-        torch.cuda.synchronize(dev)
         n_e2e = max(1, args.e2e_steps)
-        e0.record(stream)
-        for _ in range(n_e2e):
-            e2e_step()
-        e1.record(stream)
-        torch.cuda.synchronize(dev)
-        ms_e2e = ranks.max_over_ranks(e0.elapsed_time(e1) / n_e2e, dist, dev)
-        nb = lambda *ts: sum(t.numel() * t.element_size() for t in ts)
+        ms_e2e = ranks.max_over_ranks(
+            pipelined_e2e(dev, host_in, dev_in, dev_out, host_out, run, n_e2e, dist), dist, dev)
+        fa.check_device_errors(dev)
+        nb = lambda ts: sum(t.numel() * t.element_size() for t in ts)
         e2e = {"value": ranks.weak_scaling_rate(flops, world, ms_e2e) / 1e12, "unit": UNIT,
-               "h2d_bytes_per_step": nb(*hin), "d2h_bytes_per_step": nb(ho, hlse),
+               "h2d_bytes_per_step": nb(host_in), "d2h_bytes_per_step": nb(host_out),
                "steps": n_e2e, "ms_per_step": ms_e2e,
+               "pipeline": "two buffer sets; uploads and downloads overlap the kernels",
                "api": "tiled_attention_20_b200.fa.fwd_fp8 (C ABI)"}
 
     cpu = None
