@@ -284,11 +284,11 @@ __global__ void __launch_bounds__(kDecThreads) fa_decode_kernel(const DecodePara
   // Pass 2: o = sum_j p_j v_j.  Warp w takes keys w, w + 8, ... of a tile;
   // lane l holds columns [CPL*l, CPL*l + CPL).
   constexpr int CPL = D / 32;
-  float o_acc[NQP][CPL];
+  float2 o_acc[NQP][CPL / 2];
 #pragma unroll
   for (int qi = 0; qi < NQP; ++qi)
 #pragma unroll
-    for (int c = 0; c < CPL; ++c) o_acc[qi][c] = 0.f;
+    for (int c = 0; c < CPL / 2; ++c) o_acc[qi][c] = make_float2(0.f, 0.f);
   for (int i = 0; i < T && ok; ++i) {
     const int g = T + i, s = g % S;
     if (!mbar_wait(&full[s], (g / S) & 1, p.status)) {
@@ -300,8 +300,19 @@ __global__ void __launch_bounds__(kDecThreads) fa_decode_kernel(const DecodePara
     for (int kk = warp; kk < rows; kk += 8) {
       const float* pj = sbuf + (i * kDecTileKeys + kk) * NQP;
       float pv[NQP];
+      if constexpr (NQP >= 4) {
 #pragma unroll
-      for (int qi = 0; qi < NQP; ++qi) pv[qi] = pj[qi];
+        for (int q4 = 0; q4 < NQP / 4; ++q4) {
+          const float4 t4 = reinterpret_cast<const float4*>(pj)[q4];
+          pv[4 * q4] = t4.x;
+          pv[4 * q4 + 1] = t4.y;
+          pv[4 * q4 + 2] = t4.z;
+          pv[4 * q4 + 3] = t4.w;
+        }
+      } else {
+#pragma unroll
+        for (int qi = 0; qi < NQP; ++qi) pv[qi] = pj[qi];
+      }
       float vf[CPL];
       if constexpr (CPL == 4) {
         const uint2 w = *reinterpret_cast<const uint2*>(tile + kk * D * 2 + lane * 8);
@@ -315,9 +326,12 @@ __global__ void __launch_bounds__(kDecThreads) fa_decode_kernel(const DecodePara
         vf[1] = bf16_hi(w);
       }
 #pragma unroll
-      for (int qi = 0; qi < NQP; ++qi)
+      for (int qi = 0; qi < NQP; ++qi) {
+        const float2 pp = make_float2(pv[qi], pv[qi]);
 #pragma unroll
-        for (int c = 0; c < CPL; ++c) o_acc[qi][c] = fmaf(pv[qi], vf[c], o_acc[qi][c]);
+        for (int c = 0; c < CPL / 2; ++c)
+          o_acc[qi][c] = fma2(pp, make_float2(vf[2 * c], vf[2 * c + 1]), o_acc[qi][c]);
+      }
     }
     __syncwarp();
     if (lane == 0) mbar_arrive(&empty[s]);
@@ -328,7 +342,10 @@ __global__ void __launch_bounds__(kDecThreads) fa_decode_kernel(const DecodePara
 #pragma unroll
   for (int qi = 0; qi < NQP; ++qi)
 #pragma unroll
-    for (int c = 0; c < CPL; ++c) ored[(warp * NQP + qi) * D + lane * CPL + c] = o_acc[qi][c];
+    for (int c = 0; c < CPL / 2; ++c) {
+      ored[(warp * NQP + qi) * D + lane * CPL + 2 * c] = o_acc[qi][c].x;
+      ored[(warp * NQP + qi) * D + lane * CPL + 2 * c + 1] = o_acc[qi][c].y;
+    }
   asm volatile("bar.sync 1, 256;" ::: "memory");
 
   constexpr float kLn2 = 0.6931471805599453f;
