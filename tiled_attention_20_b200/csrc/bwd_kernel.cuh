@@ -113,9 +113,9 @@ struct BwdLayout {
 // warpgroup 0 (producer, MMA issuer, two idle warps) and the drain
 // warpgroup give registers to the two compute warpgroups.
 constexpr int kBwdLaunchRegs = 128;
-constexpr int kBwdCtlRegs = 64;
-constexpr int kBwdComputeRegs = 176;
-constexpr int kBwdDrainRegs = 80;
+constexpr int kBwdCtlRegs = 72;
+constexpr int kBwdComputeRegs = 168;
+constexpr int kBwdDrainRegs = 88;
 static_assert(128 * kBwdCtlRegs + 256 * kBwdComputeRegs + 128 * kBwdDrainRegs <=
                   512 * kBwdLaunchRegs,
               "register split exceeds the launch allocation");
