@@ -94,3 +94,21 @@ def test_fp8_input_recipe():
         tol = torch.maximum(2.0 ** -4 * r.abs() + 2.0 ** -8 * r.abs(),
                             (2.0 ** -10) * f.double()[:, :, None, None])
         assert torch.all((deq - r).abs() <= tol)
+
+
+def test_decode_input_recipe():
+    """decode_qkv: seeded (same seed, same tensors), bf16, and ragged lengths
+    drawn in [L/2, L] (all L without ragged)."""
+    import torch
+    a = inputs.decode_qkv(3, 2, 4, 100, 64, seed=9, ragged=True)
+    b = inputs.decode_qkv(3, 2, 4, 100, 64, seed=9, ragged=True)
+    for x, y in zip(a, b):
+        assert torch.equal(x, y)
+    q, k, v, lens = a
+    assert q.dtype == k.dtype == v.dtype == torch.bfloat16
+    assert q.shape == (3, 2, 4, 64) and k.shape == v.shape == (3, 2, 100, 64)
+    assert lens.dtype == torch.int32 and torch.all((lens >= 50) & (lens <= 100))
+    _, _, _, full = inputs.decode_qkv(3, 2, 4, 100, 64, seed=9)
+    assert torch.all(full == 100)
+    for w in (inputs.DECODE_B8, inputs.DECODE_B8_RAGGED, inputs.DECODE_SPEC, inputs.DECODE_LONG):
+        assert 1 <= w.Nq <= 8 and w.d in (64, 128)
