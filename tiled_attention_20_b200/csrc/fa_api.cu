@@ -1,7 +1,8 @@
 // fa_api.cu -- the C ABI of libfa (declared in include/fa.h): argument
-// validation, TMA descriptor construction, persistent-grid sizing and kernel
-// launches.  Every step of the computation runs in the kernels; this file
-// only prepares launches.
+// validation, TMA descriptor construction, persistent-grid and split
+// planning, and kernel launches.  Every step of the computation runs in the
+// kernels (the *_kernel.cuh headers); this file only prepares launches, and
+// holds the one-thread kernel of the failure-detection self-test.
 #include <cfloat>
 #include <cmath>
 #include <cstdint>
