@@ -15,7 +15,6 @@ HERE = os.path.dirname(os.path.abspath(__file__))
 CSRC = os.path.join(HERE, "csrc")
 LIB = os.path.join(HERE, "libfa.so")
 SOURCES = ["fa_api.cu"]
-DEPS = ["fa_api.cu", "fwd_kernel.cuh", "bwd_kernel.cuh", "dq_kernel.cuh", "decode_kernel.cuh", "sm100.cuh"]
 HEADER = os.path.join(os.path.dirname(HERE), "include", "fa.h")
 
 NVCC_FLAGS = [
@@ -37,7 +36,9 @@ def stale() -> bool:
     if not os.path.exists(LIB):
         return True
     t = os.path.getmtime(LIB)
-    deps = [os.path.join(CSRC, f) for f in DEPS] + [HEADER]
+    # every source and header of the single translation unit, plus the C header
+    deps = [os.path.join(CSRC, f) for f in os.listdir(CSRC) if f.endswith((".cu", ".cuh"))]
+    deps.append(HEADER)
     return any(os.path.getmtime(p) > t for p in deps)
 
 
