@@ -157,7 +157,29 @@ int check_scale(float scale) {
 
 int make_tmap_rows(CUtensorMap* m, const void* base, int BH, int N, int d, int box_rows);
 
-int fwd_units(int B, int H, int N) { return B * H * ((N + 255) / 256); }
+// Forward schedule (fwd_item).  Causal heads with an even number P >= 8 of
+// tile pairs are dealt as merged complementary pairs, except for the last
+// R = (P / 2) << shift heads, left as single pairs; shift is the smallest
+// that gives those at least two rounds of the persistent grid.  Returns h1
+// (the number of merged heads) and sets the decode's divisor and shift.
+int fwd_schedule(int BH, int N, int causal, int sms, int* item_div, int* tail_shift) {
+  const int P = (N + 255) / 256;
+  *item_div = BH;
+  *tail_shift = 0;
+  if (!causal || P < 8 || (P & 1)) return 0;
+  const int half = P / 2;
+  int shift = 0;
+  while ((static_cast<long long>(half) << shift) * P < 2LL * sms) ++shift;
+  const long long R = static_cast<long long>(half) << shift;
+  if (BH <= R) return 0;
+  *item_div = half;
+  *tail_shift = shift;
+  return BH - static_cast<int>(R);
+}
+int fwd_items(int BH, int N, int h1) {
+  const int P = (N + 255) / 256;
+  return h1 * (P / 2) + (BH - h1) * P;  // h1 > 0 only when P is even
+}
 
 template <int D, bool CAUSAL, bool FP8 = false>
 int launch_fwd(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
@@ -634,14 +656,16 @@ int fa_decode(const void* q, const void* k_cache, const void* v_cache, void* o, 
 }
 
 int fa_launch_shape(int pass, int B, int H, int N, int d, int causal, int* ctas, int* work_units) {
-  (void)causal;
   if (!ctas || !work_units) return FA_ERR_NULL;
   int s = check_shape(B, H, N, d);
   if (s != FA_OK) return s;
   DeviceInfo* info = nullptr;
   s = device_info(&info);
   if (s != FA_OK) return s;
-  const int units = pass == 0 ? fwd_units(B, H, N) : fa::bwd_units(B, H, N);
+  int item_div, tail_shift;
+  const int units =
+      pass == 0 ? fwd_items(B * H, N, fwd_schedule(B * H, N, causal, info->sms, &item_div, &tail_shift))
+                : fa::bwd_units(B, H, N);
   *work_units = units;
   *ctas = units < info->sms ? units : info->sms;
   return FA_OK;
@@ -670,7 +694,8 @@ int fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int
   p.BH = BH;
   p.N = N;
   p.n_qt2 = (N + 255) / 256;
-  p.n_units = fwd_units(B, H, N);
+  p.h1 = fwd_schedule(BH, N, causal, info->sms, &p.item_div, &p.tail_shift);
+  p.n_units = fwd_items(BH, N, p.h1);
   // Masked scores are -inf before scaling; a zero scale would turn them into
   // NaN.  FLT_MIN keeps them at -inf while every finite score still scales
   // to zero, so scale = 0 gives exactly uniform weights.
@@ -780,7 +805,8 @@ int fa_fwd_fp8(const void* q, const void* k, const void* v, const float* descale
   p.BH = BH;
   p.N = N;
   p.n_qt2 = (N + 255) / 256;
-  p.n_units = fwd_units(B, H, N);
+  p.h1 = fwd_schedule(BH, N, causal, info->sms, &p.item_div, &p.tail_shift);
+  p.n_units = fwd_items(BH, N, p.h1);
   p.scale_log2 = scale * 1.4426950408889634f;  // the kernel folds in the descales, then clamps
   p.status = info->status;
   const int ctas = p.n_units < info->sms ? p.n_units : info->sms;

@@ -58,7 +58,10 @@ struct FwdParams {
   int BH;
   int N;
   int n_qt2;       // ceil(N / 256): Q tile pairs per head
-  int n_units;     // BH * n_qt2
+  int n_units;     // scheduling items (fwd_item): BH * n_qt2 when h1 == 0
+  int h1;          // causal: heads whose tile pairs are dealt two at a time
+  int item_div;    // causal: n_qt2 / 2 if h1 > 0, else BH
+  int tail_shift;  // causal: the single-pair heads number item_div << tail_shift
   float scale_log2;  // scale * log2(e)
   int* status;
 };
@@ -94,39 +97,73 @@ struct FwdBarriers {
   uint64_t mma_done;
   uint32_t tmem_base;
   int abort_flag;
+  int unit_nk[2][2];  // key tiles of the two Q tiles of the n-th unit, slot n & 1
 };
+static_assert(sizeof(FwdBarriers) <= FwdLayout<64>::kBarBytes, "barrier block overflows its slot");
 
 struct FwdUnit {
   int bh, q0, nk0, nk1;
 };
 
-// Work unit w -> (head, Q tile pair).  Causal: tile-pair index major, head
-// minor, so units come longest first across all heads (load balance).
-// Non-causal (all units equal): heads in groups of kUnitHeadGroup, tile
-// pair major within a group, so the CTAs running at one time share a few
-// heads' K and V in L2 instead of streaming every head's.
+// One Q tile pair of one head: its first row and the key tiles each of its
+// two Q tiles reads (all of them, or up to the diagonal when causal).
+__device__ __forceinline__ FwdUnit fwd_pair(const FwdParams& p, int bh, int qt2, bool causal) {
+  FwdUnit u;
+  u.bh = bh;
+  u.q0 = qt2 * 256;
+  const int nkv = (p.N + 127) / 128;
+  u.nk0 = causal ? min(2 * qt2 + 1, nkv) : nkv;
+  u.nk1 = causal ? min(2 * qt2 + 2, nkv) : nkv;
+  return u;
+}
+
+// Non-causal items (all equal): one tile pair each, heads in groups of
+// kUnitHeadGroup, tile pair major within a group, so the CTAs running at
+// one time share a few heads' K and V in L2 instead of streaming every
+// head's.
 constexpr int kUnitHeadGroup = 8;
 
+// Causal scheduling items.  Tile pair t of a head costs about 4t + 3 key
+// tiles, so pairs t and n_qt2 - 1 - t together cost the same for every t.
+// The first h1 heads are dealt as such merged items, head-major: every item
+// costs the same, and the CTAs running at one time share a few heads' K and
+// V in L2 instead of streaming every head's.  The other R heads follow as
+// single pairs, longest first across heads, so the snake's last rounds even
+// out the per-CTA totals.  With merging (n_qt2 even), R = (n_qt2 / 2) <<
+// tail_shift, so one division by item_div decodes both kinds of item; h1 = 0
+// (item_div = BH, tail_shift = 0) is the plain longest-first order.  Item w
+// holds one or two pairs; sets u to pair `sub` and returns true if it exists.
 template <bool CAUSAL>
-__device__ __forceinline__ FwdUnit fwd_decode(const FwdParams& p, int w) {
-  FwdUnit u;
-  int idx;
-  if (CAUSAL) {
-    idx = w / p.BH;
-    u.bh = w - idx * p.BH;
-  } else {
+__device__ __forceinline__ bool fwd_item(const FwdParams& p, int w, int sub, FwdUnit& u) {
+  if (w < 0) return false;
+  if (!CAUSAL) {
+    if (sub) return false;
     const int g = w / (kUnitHeadGroup * p.n_qt2), g0 = g * kUnitHeadGroup;
     const int gs = min(kUnitHeadGroup, p.BH - g0);
     const int r = w - g * kUnitHeadGroup * p.n_qt2;  // every earlier group is full
-    idx = r / gs;
-    u.bh = g0 + (r - idx * gs);
+    const int idx = r / gs;
+    u = fwd_pair(p, g0 + (r - idx * gs), idx, false);
+    return true;
   }
-  const int qt2 = CAUSAL ? (p.n_qt2 - 1 - idx) : idx;
-  u.q0 = qt2 * 256;
-  const int nkv = (p.N + 127) / 128;
-  u.nk0 = CAUSAL ? min(2 * qt2 + 1, nkv) : nkv;
-  u.nk1 = CAUSAL ? min(2 * qt2 + 2, nkv) : nkv;
-  return u;
+  const int d = p.item_div, n1 = p.h1 * d, P = p.n_qt2;
+  const bool merged = w < n1;
+  if (sub && !merged) return false;
+  const int w2 = merged ? w : w - n1;
+  const int q = w2 / d;
+  if (merged) {
+    const int k = w2 - q * d;
+    u = fwd_pair(p, q, sub ? k : P - 1 - k, true);
+  } else {
+    const int idx = q >> p.tail_shift;  // = w2 / R
+    u = fwd_pair(p, p.h1 + w2 - ((idx * d) << p.tail_shift), P - 1 - idx, true);
+  }
+  return true;
+}
+
+// Whether item w has a pair `sub` (fwd_item without the decode).
+template <bool CAUSAL>
+__device__ __forceinline__ bool fwd_item_exists(const FwdParams& p, int w, int sub) {
+  return w >= 0 && (!sub || (CAUSAL && w < p.h1 * p.item_div));
 }
 
 // Static "snake" assignment of work units to persistent CTAs: in round r,
@@ -172,11 +209,15 @@ __device__ void fwd_producer(const CUtensorMap* tm_q, const CUtensorMap* tm_k,
   // A tile is D/64 boxes of 64 bf16 columns, or one box of 128 E4M3 columns;
   // either way a box row is 128 bytes.
   constexpr int NB = FP8 ? 1 : D / 64;
-  for (int r = 0, nr = snake_rounds(p.n_units); r < nr; ++r) {
-    const int w = snake_unit(r, p.n_units);
-    if (w < 0) continue;
-    const FwdUnit u = fwd_decode<CAUSAL>(p, w);
+  for (int it = 0, ni = 2 * snake_rounds(p.n_units); it < ni; ++it) {
+    FwdUnit u;
+    if (!fwd_item<CAUSAL>(p, snake_unit(it >> 1, p.n_units), it & 1, u)) continue;
     if (units > 0 && !wait1(&b->q_empty, (units - 1) & 1, b, p.status)) return;
+    // The MMA issuer reads the unit's key-tile counts after its q_full wait
+    // (the arrival below releases these stores); slot units & 1 was last read
+    // two units ago, before that unit's Q tiles were released.
+    *(volatile int*)&b->unit_nk[units & 1][0] = u.nk0;
+    *(volatile int*)&b->unit_nk[units & 1][1] = u.nk1;
     mbar_arrive_expect_tx(&b->q_full, 2 * L::kTileBytes);
     ++units;  // number of times q_full has been armed
 #pragma unroll
@@ -282,12 +323,11 @@ __device__ void fwd_mma(const FwdParams& p, uint8_t* smem, FwdBarriers* b, uint3
   const uint32_t qs[2] = {sb + L::kQ0, sb + L::kQ1};
   int qc = 0, kc = 0, vc = 0;
   int pc[2] = {0, 0};
-  for (int r = 0, nr = snake_rounds(p.n_units); r < nr; ++r) {
-    const int w = snake_unit(r, p.n_units);
-    if (w < 0) continue;
-    const FwdUnit u = fwd_decode<CAUSAL>(p, w);
-    const int nk0 = u.nk0, nk1 = u.nk1, nk = u.nk1;
+  for (int it = 0, ni = 2 * snake_rounds(p.n_units); it < ni; ++it) {
+    if (!fwd_item_exists<CAUSAL>(p, snake_unit(it >> 1, p.n_units), it & 1)) continue;
     if (!wait1(&b->q_full, qc & 1, b, p.status)) return;
+    const int nk0 = *(volatile int*)&b->unit_nk[qc & 1][0];
+    const int nk1 = *(volatile int*)&b->unit_nk[qc & 1][1], nk = nk1;
     ++qc;
     tc_fence_after();
     for (int j = 0; j < nk; ++j) {
@@ -404,10 +444,9 @@ __device__ void fwd_softmax(const FwdParams& p, FwdBarriers* b, uint32_t tmem, i
   const uint32_t tO = tmem + lane_base + 256u + wg * D;
   const int N = p.N;
   int sc = 0, oc = 0;
-  for (int r = 0, nr = snake_rounds(p.n_units); r < nr; ++r) {
-    const int w = snake_unit(r, p.n_units);
-    if (w < 0) continue;
-    const FwdUnit u = fwd_decode<CAUSAL>(p, w);
+  for (int it = 0, ni = 2 * snake_rounds(p.n_units); it < ni; ++it) {
+    FwdUnit u;
+    if (!fwd_item<CAUSAL>(p, snake_unit(it >> 1, p.n_units), it & 1, u)) continue;
     const int nk = wg ? u.nk1 : u.nk0;
     const int tile_row0 = u.q0 + wg * 128;
     const int row = tile_row0 + t;
