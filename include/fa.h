@@ -171,7 +171,10 @@ int fa_selftest_wait_timeout(int limit_ms, fa_stream_t stream);
 
 /* Number of persistent CTAs fa_fwd / fa_bwd launch for a problem on the
  * current device (pass = 0 forward, 1 backward), and the number of work
- * units they share; for the harness and its wave-quantization checks.
+ * units they share (forward: scheduling items, each one Q tile pair, or
+ * for causal problems with an even number >= 8 of tile pairs per head
+ * mostly two complementary pairs of one head; backward: K/V blocks);
+ * for the harness and its wave-quantization checks.
  * Returns FA_OK or an error status (no launch happens). */
 int fa_launch_shape(int pass, int B, int H, int N, int d, int causal,
                     int *ctas, int *work_units);
