@@ -1,6 +1,5 @@
 """The C ABI without a GPU: the library loads, exports every symbol the header
 declares, and rejects bad arguments before touching the device."""
-import ctypes
 import os
 import re
 

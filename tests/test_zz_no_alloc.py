@@ -6,7 +6,6 @@ results must match fa_bwd's.
 
 This file is named to be collected last, so that a run stopping at the first
 failure has already run every other test."""
-import ctypes
 
 import pytest
 import torch
