@@ -179,6 +179,21 @@ int fa_selftest_wait_timeout(int limit_ms, fa_stream_t stream);
 int fa_launch_shape(int pass, int B, int H, int N, int d, int causal,
                     int *ctas, int *work_units);
 
+/* Work-unit schedule of fa_fwd / fa_fwd_fp8 on a device with `sms` SMs (host
+ * arithmetic, no device needed).  A head of N queries has P = ceil(N/256)
+ * Q tile pairs; a causal pair t costs about 4t + 3 key tiles, so pairs t and
+ * P-1-t cost the same together for every t.  When the problem is causal and
+ * P is even and >= 8, the first *merged_heads heads are dealt as items of
+ * two such complementary pairs (head-major, so running CTAs share a few
+ * heads' K and V in L2) and the last R = (P/2) << *tail_shift heads as single
+ * pairs, longest first, with *tail_shift the smallest shift giving R * P >=
+ * 2 * sms (two rounds of the persistent grid).  Otherwise, and when
+ * B*H <= R, every item is one pair (*merged_heads = 0, *tail_shift = 0).  *items = merged_heads * P/2 + (B*H - merged_heads) * P
+ * items are dealt to min(*items, sms) CTAs.  B, H, N, sms >= 1 and
+ * B*H*P < 2^31, else FA_ERR_SHAPE; FA_ERR_NULL for a NULL output. */
+int fa_fwd_schedule(int B, int H, int N, int causal, int sms, int *items,
+                    int *merged_heads, int *tail_shift);
+
 /*
  * Decode: attention of Nq new queries per head against a key/value cache
  * ("第17讲 Tensor Core、HBM、SRAM 与 FlashAttention", §9.2 prefill and decode,

@@ -52,6 +52,14 @@ int main(void) {
       bad = 1;
     }
   }
+  {
+    int items = 0, merged = 0, shift = 0;
+    bad |= expect("fwd schedule", fa_fwd_schedule(2, 32, 4096, 1, 148, &items, &merged, &shift), FA_OK);
+    if (items != 32 * 8 + 32 * 16 || merged != 32 || shift != 2) {
+      printf("  %d items, %d merged heads, shift %d; expected 768, 32, 2\n", items, merged, shift);
+      bad = 1;
+    }
+  }
   printf(bad ? "FAILED\n" : "OK\n");
   return bad;
 }

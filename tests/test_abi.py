@@ -155,6 +155,56 @@ def test_gemm_tiles(lib):
         fa.gemm_tiles(0, 5, 148)
 
 
+def test_fwd_schedule_values(lib):
+    """Causal B=2 H=32 N=4096: 16 tile pairs per head; the single-pair tail
+    needs R * 16 >= 2 * 148, R = 8 << s, so s = 2 and R = 32: 32 heads of 8
+    merged items and 32 heads of 16 single pairs.  B=8 H=16 N=8192: 32 pairs,
+    R = 16 (16 * 32 = 512 >= 296), 112 merged heads.  No merging for
+    non-causal problems, an odd pair count, fewer than 8 pairs, or heads not
+    outnumbering the tail."""
+    import tiled_attention_20_b200.fa as fa
+    assert fa.fwd_schedule(2, 32, 4096, True) == (32 * 8 + 32 * 16, 32, 2)
+    assert fa.fwd_schedule(8, 16, 8192, True) == (112 * 16 + 16 * 32, 112, 0)
+    assert fa.fwd_schedule(2, 32, 4096, False) == (64 * 16, 0, 0)
+    assert fa.fwd_schedule(2, 20, 2300, True) == (40 * 9, 0, 0)      # 9 pairs: odd
+    assert fa.fwd_schedule(16, 16, 1024, True) == (256 * 4, 0, 0)    # 4 pairs
+    assert fa.fwd_schedule(1, 16, 16384, True) == (16 * 64, 0, 0)    # 16 heads <= R = 32
+    assert fa.fwd_schedule(1, 16, 6656, True) == (3 * 13 + 13 * 26, 3, 0)
+    with pytest.raises(fa.FAError):
+        fa.fwd_schedule(0, 1, 256, True)
+    with pytest.raises(fa.FAError):
+        fa.fwd_schedule(1, 1, 256, True, sms=0)
+
+
+def test_fwd_schedule_rule(lib):
+    """The defining properties of the schedule over many shapes and SM
+    counts: merging only for causal problems with an even pair count P >= 8;
+    the single-pair tail is R = (P/2) << s heads with s the smallest shift
+    giving R * P >= 2 * sms; the item count adds up."""
+    import tiled_attention_20_b200.fa as fa
+    for sms in (1, 7, 108, 132, 148):
+        for BH in (1, 3, 8, 16, 33, 64, 100, 128, 257):
+            for N in (1, 256, 1792, 1793, 2048, 2300, 4000, 4096, 6656, 8192, 16384):
+                P = (N + 255) // 256
+                for causal in (False, True):
+                    items, h1, s = fa.fwd_schedule(1, BH, N, causal, sms)
+                    eligible = causal and P >= 8 and P % 2 == 0
+                    if not eligible:
+                        assert (items, h1, s) == (BH * P, 0, 0)
+                        continue
+                    half = P // 2
+                    s_min = 0
+                    while (half << s_min) * P < 2 * sms:
+                        s_min += 1
+                    assert s == (s_min if h1 else 0)
+                    R = half << s_min
+                    assert h1 == (BH - R if BH > R else 0)
+                    assert items == h1 * half + (BH - h1) * P
+                    if h1:
+                        assert (half << s) * P >= 2 * sms
+                        assert s == 0 or (half << (s - 1)) * P < 2 * sms
+
+
 def test_selftest_limit_validation(lib):
     assert lib.fa_selftest_wait_timeout(0, None) == -10
     assert lib.fa_selftest_wait_timeout(2001, None) == -10

@@ -671,6 +671,19 @@ int fa_launch_shape(int pass, int B, int H, int N, int d, int causal, int* ctas,
   return FA_OK;
 }
 
+int fa_fwd_schedule(int B, int H, int N, int causal, int sms, int* items, int* merged_heads,
+                    int* tail_shift) {
+  if (!items || !merged_heads || !tail_shift) return FA_ERR_NULL;
+  if (B < 1 || H < 1 || N < 1 || sms < 1 ||
+      static_cast<long long>(B) * H * ((N + 255) / 256) >= (1LL << 31))
+    return FA_ERR_SHAPE;
+  int item_div = 0;
+  const int h1 = fwd_schedule(B * H, N, causal, sms, &item_div, tail_shift);
+  *merged_heads = h1;
+  *items = fwd_items(B * H, N, h1);
+  return FA_OK;
+}
+
 int fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int N,
            int d, float scale, int causal, fa_stream_t stream) {
   if (!q || !k || !v || !o || !lse) return FA_ERR_NULL;

@@ -29,7 +29,8 @@ EXPORTED = ["fa_fwd", "fa_bwd", "fa_bwd_workspace_size", "fa_strerror",
             "fa_check_device_errors", "fa_launch_shape", "fa_trace_start", "fa_trace_stop",
             "fa_trace_kernel_name", "fa_bwd_noalloc", "fa_bwd_deterministic",
             "fa_decode", "fa_decode_workspace_size", "fa_decode_plan", "fa_fwd_fp8",
-            "fa_gemm", "fa_gemm_workspace_size", "fa_gemm_tiles", "fa_selftest_wait_timeout"]
+            "fa_gemm", "fa_gemm_workspace_size", "fa_gemm_tiles", "fa_selftest_wait_timeout",
+            "fa_fwd_schedule"]
 NOALLOC_MAX_SCRATCH = 32 << 20  # FA_BWD_NOALLOC_MAX_SCRATCH
 KERNEL_IDS = {0: "fa_fwd_kernel", 1: "fa_bwd_prep", 2: "fa_bwd_kernel", 3: "fa_bwd_dq_convert",
               4: "fa_dq_kernel", 5: "fa_decode_kernel", 6: "fa_gemm_kernel", 7: "fa_gemm_pack"}
@@ -89,6 +90,9 @@ def load(path: str = LIB_PATH):
         lib.fa_gemm_tiles.argtypes = [_i, _i, _i, ctypes.POINTER(_i), ctypes.POINTER(_i),
                                       ctypes.POINTER(_i)]
         lib.fa_gemm_tiles.restype = _i
+        lib.fa_fwd_schedule.argtypes = [_i, _i, _i, _i, _i, ctypes.POINTER(_i),
+                                         ctypes.POINTER(_i), ctypes.POINTER(_i)]
+        lib.fa_fwd_schedule.restype = _i
         lib.fa_fwd_fp8.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _f,
                                    _i, _vp]
         lib.fa_fwd_fp8.restype = _i
@@ -330,6 +334,14 @@ def gemm_tiles(M, N, sms=148):
     _check(load().fa_gemm_tiles(M, N, sms, ctypes.byref(bn), ctypes.byref(tm), ctypes.byref(tn)),
            "fa_gemm_tiles")
     return bn.value, tm.value, tn.value
+
+
+def fwd_schedule(B, H, N, causal=False, sms=148):
+    """(items, merged_heads, tail_shift) of fa_fwd's work-unit schedule."""
+    items, merged, shift = _i(0), _i(0), _i(0)
+    _check(load().fa_fwd_schedule(B, H, N, int(bool(causal)), sms, ctypes.byref(items),
+                                  ctypes.byref(merged), ctypes.byref(shift)), "fa_fwd_schedule")
+    return items.value, merged.value, shift.value
 
 
 def _ld(t):
