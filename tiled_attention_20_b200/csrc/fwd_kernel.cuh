@@ -18,10 +18,11 @@
 // the A operand of O_i += P_i V straight from TMEM.  One thread owns one row,
 // so row max and row sum need no shuffles.
 //
-// A work unit is (b*H+h, pair of 128-row Q tiles); units are sorted longest
-// first when causal and dealt to a persistent grid of min(units, SMs) CTAs
-// in a snake order, so no partial last wave of whole CTAs is left (wave
+// A work unit is (b*H+h, pair of 128-row Q tiles).  Scheduling items of one
+// or two units are dealt to a persistent grid of min(items, SMs) CTAs in a
+// snake order, so no partial last wave of whole CTAs is left (wave
 // quantization, "CS336 Lecture 5 · GPUs, TPUs" notes, section "波次量化").
+// Causal items pair complementary tile pairs of one head (fwd_item).
 //
 // Causal masking is by tile skipping: Q tile i only visits key tiles up to
 // its diagonal, and only the diagonal tile (and a ragged last key tile) pays
