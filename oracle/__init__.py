@@ -36,54 +36,63 @@ _dp = ctypes.POINTER(ctypes.c_double)
 _ip = ctypes.POINTER(ctypes.c_int)
 
 
+def compile_source(src: str, out: str) -> str:
+    """gcc a copy of the oracle's C source into a shared library."""
+    tmp = out + ".tmp%d" % os.getpid()
+    subprocess.check_call(
+        ["gcc", "-O2", "-fopenmp", "-fPIC", "-shared", "-std=c11", "-o", tmp, src, "-lm"])
+    os.replace(tmp, out)
+    return out
+
+
 def build(force: bool = False) -> str:
     """Compile the oracle with gcc into ``oracle/liboracle.so``."""
     if force or not os.path.exists(_LIB) or os.path.getmtime(_LIB) < os.path.getmtime(_SRC):
-        tmp = _LIB + ".tmp%d" % os.getpid()
-        subprocess.check_call(
-            ["gcc", "-O2", "-fopenmp", "-fPIC", "-shared", "-std=c11",
-             "-o", tmp, _SRC, "-lm"])
-        os.replace(tmp, _LIB)
+        compile_source(_SRC, _LIB)
     return _LIB
 
 
 _lib = None
 
 
+def bind(lib):
+    """Declare the C signatures on a loaded copy of the oracle library."""
+    lib.oracle_fwd.argtypes = [_dp, _dp, _dp, ctypes.c_int, ctypes.c_int, ctypes.c_int,
+                               ctypes.c_int, ctypes.c_double, ctypes.c_int, _dp, _dp]
+    lib.oracle_fwd.restype = None
+    lib.oracle_fwd_rows.argtypes = [_dp, _dp, _dp, ctypes.c_int, ctypes.c_int,
+                                    ctypes.c_double, ctypes.c_int, _ip, ctypes.c_int,
+                                    _dp, _dp]
+    lib.oracle_fwd_rows.restype = None
+    lib.oracle_probs.argtypes = [_dp, _dp, ctypes.c_int, ctypes.c_int, ctypes.c_double,
+                                 ctypes.c_int, _dp]
+    lib.oracle_probs.restype = None
+    lib.oracle_bwd.argtypes = [_dp, _dp, _dp, _dp, ctypes.c_int, ctypes.c_int, ctypes.c_int,
+                               ctypes.c_int, ctypes.c_double, ctypes.c_int, _dp, _dp, _dp, _dp]
+    lib.oracle_bwd.restype = ctypes.c_double
+    lib.oracle_online_fwd.argtypes = [_dp, _dp, _dp, ctypes.c_int, ctypes.c_int,
+                                      ctypes.c_double, ctypes.c_int, ctypes.c_int, _dp, _dp]
+    lib.oracle_online_fwd.restype = None
+    lib.oracle_loss.argtypes = [_dp, _dp, _dp, _dp, ctypes.c_int, ctypes.c_int,
+                                ctypes.c_double, ctypes.c_int]
+    lib.oracle_loss.restype = ctypes.c_double
+    lib.oracle_decode.argtypes = [_dp, _dp, _dp, _ip, ctypes.c_int, ctypes.c_int,
+                                  ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_double,
+                                  ctypes.c_int, _dp, _dp]
+    lib.oracle_decode.restype = None
+    lib.oracle_gemm.argtypes = [_dp, _dp, _dp, ctypes.c_int, ctypes.c_int, ctypes.c_int]
+    lib.oracle_gemm.restype = None
+    lib.oracle_num_threads.argtypes = []
+    lib.oracle_num_threads.restype = ctypes.c_int
+    lib.oracle_set_num_threads.argtypes = [ctypes.c_int]
+    lib.oracle_set_num_threads.restype = None
+    return lib
+
+
 def _load():
     global _lib
     if _lib is None:
-        lib = ctypes.CDLL(build())
-        lib.oracle_fwd.argtypes = [_dp, _dp, _dp, ctypes.c_int, ctypes.c_int, ctypes.c_int,
-                                   ctypes.c_int, ctypes.c_double, ctypes.c_int, _dp, _dp]
-        lib.oracle_fwd.restype = None
-        lib.oracle_fwd_rows.argtypes = [_dp, _dp, _dp, ctypes.c_int, ctypes.c_int,
-                                        ctypes.c_double, ctypes.c_int, _ip, ctypes.c_int,
-                                        _dp, _dp]
-        lib.oracle_fwd_rows.restype = None
-        lib.oracle_probs.argtypes = [_dp, _dp, ctypes.c_int, ctypes.c_int, ctypes.c_double,
-                                     ctypes.c_int, _dp]
-        lib.oracle_probs.restype = None
-        lib.oracle_bwd.argtypes = [_dp, _dp, _dp, _dp, ctypes.c_int, ctypes.c_int, ctypes.c_int,
-                                   ctypes.c_int, ctypes.c_double, ctypes.c_int, _dp, _dp, _dp, _dp]
-        lib.oracle_bwd.restype = ctypes.c_double
-        lib.oracle_online_fwd.argtypes = [_dp, _dp, _dp, ctypes.c_int, ctypes.c_int,
-                                          ctypes.c_double, ctypes.c_int, ctypes.c_int, _dp, _dp]
-        lib.oracle_online_fwd.restype = None
-        lib.oracle_loss.argtypes = [_dp, _dp, _dp, _dp, ctypes.c_int, ctypes.c_int,
-                                    ctypes.c_double, ctypes.c_int]
-        lib.oracle_loss.restype = ctypes.c_double
-        lib.oracle_decode.argtypes = [_dp, _dp, _dp, _ip, ctypes.c_int, ctypes.c_int,
-                                      ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_double,
-                                      ctypes.c_int, _dp, _dp]
-        lib.oracle_decode.restype = None
-        lib.oracle_gemm.argtypes = [_dp, _dp, _dp, ctypes.c_int, ctypes.c_int, ctypes.c_int]
-        lib.oracle_gemm.restype = None
-        lib.oracle_num_threads.argtypes = []
-        lib.oracle_num_threads.restype = ctypes.c_int
-        lib.oracle_set_num_threads.argtypes = [ctypes.c_int]
-        lib.oracle_set_num_threads.restype = None
-        _lib = lib
+        _lib = bind(ctypes.CDLL(build()))
     return _lib
 
 
