@@ -240,6 +240,55 @@ class ClockSampler:
                 "samples": len(rows)}
 
 
+# ---------------------------------------------------------------- timing
+def timed_passes(step, steps, stream, dev, dist, world):
+    """Three timed passes of `step` on `stream`, each bracketed by a barrier
+    and a synchronize:
+      1. the headline: `steps` steps back to back between two CUDA events,
+         nothing else on the stream (so consecutive kernels may overlap their
+         boundaries); returns the mean step time, max over ranks;
+      2. the distribution: max(100, steps) steps with an event after each,
+         for the median, 10th and 90th percentile of the step time;
+      3. the per-kernel trace: `steps` steps with every library launch
+         bracketed by events (fa.trace_start / trace_stop).
+    Returns (mean ms, stats dict, traced kernels)."""
+    import tiled_attention_20_b200.fa as fa
+
+    def sync():
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize(dev)
+
+    sync()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(steps):
+        step()
+    e1.record(stream)
+    sync()
+    ms = ranks.max_over_ranks(e0.elapsed_time(e1) / steps, dist, dev)
+
+    n = max(100, steps)
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(n + 1)]
+    ev[0].record(stream)
+    for i in range(n):
+        step()
+        ev[i + 1].record(stream)
+    sync()
+    per = sorted(ev[i].elapsed_time(ev[i + 1]) for i in range(n))
+    pick = lambda f: per[min(n - 1, int(round(f * (n - 1))))]
+    stats = {"n": n, "median_ms": statistics.median(per), "p10_ms": pick(0.1),
+             "p90_ms": pick(0.9), "min_ms": per[0], "max_ms": per[-1]}
+
+    fa.trace_start()
+    for _ in range(steps):
+        step()
+    sync()
+    traced = fa.trace_stop()
+    return ms, stats, traced
+
+
 # ---------------------------------------------------------------- CPU oracle
 def cpu_oracle_rate(q, k, v, dO, w, seconds: float):
     """The oracle (fp64, as it stands) on whole heads of the workload until
@@ -349,25 +398,12 @@ def run_ours(args, rank, world, local_rank, dist):
     # keep the GPU busy while the sampler starts, outside the timed region
     for _ in range(max(3, args.warmup)):
         step()
-    if world > 1:
-        dist.barrier()
-    torch.cuda.synchronize(dev)
-    e0 = torch.cuda.Event(enable_timing=True)
-    e1 = torch.cuda.Event(enable_timing=True)
-    fa.trace_start()
-    e0.record(stream)
-    for _ in range(args.steps):
-        step()
-    e1.record(stream)
-    torch.cuda.synchronize(dev)
-    traced = fa.trace_stop()
-    if world > 1:
-        dist.barrier()
+    ms, stats, traced = timed_passes(step, args.steps, stream, dev, dist, world)
     clocks = sampler.stop()
     fa.check_device_errors(dev)
-    ms = ranks.max_over_ranks(e0.elapsed_time(e1) / args.steps, dist, dev)
     flops = step_flops(w)
     value = ranks.weak_scaling_rate(flops, world, ms) / 1e12
+    stats["tflops_at_median"] = flops / (stats["median_ms"] * 1e-3) / 1e12
 
     # dominant kernel by traced time
     dom = max(traced.items(), key=lambda kv: kv[1][1])
@@ -442,7 +478,7 @@ def run_ours(args, rank, world, local_rank, dist):
                                           "bwd": "deterministic" if args.deterministic else "atomic_dq"}),
             "pct_of_peak": value / world / peaks["bf16_tflops"],
             "roofline": roof, "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": gpu_launches,
-            "kernels": kernels, "clocks": clocks,
+            "kernels": kernels, "clocks": clocks, "step_stats": stats,
         }
         print(json.dumps(line), flush=True)
 

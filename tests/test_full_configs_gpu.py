@@ -8,6 +8,7 @@ causal row 0 equals V_0 bit for bit and its lse equals scale*q_0.k_0, the
 gradient sum rules (sum_j dK_j = 0, sum_j dV_j = sum_i dO_i) hold within the
 kernel's rounding bounds, and the outputs are finite."""
 import math
+import random
 
 import numpy as np
 import pytest
@@ -15,7 +16,7 @@ import torch
 
 import oracle
 from tiled_attention_20_b200 import inputs
-from tests.parity import assert_close, assert_close_scaled, np64
+from tests.parity import assert_close, assert_close_bf16_out, max_abs, np64, record
 
 pytestmark = pytest.mark.gpu
 DEV = "cuda:0"
@@ -26,30 +27,40 @@ def _fa():
     return fa
 
 
-def _run(w):
+def _run(w, grad_f32=False):
+    """Forward and backward of workload w on the GPU: (inputs, (o, lse, dq,
+    dk, dv)) on the CPU, plus, with grad_f32, the gradients again with fp32
+    outputs from the same forward."""
     fa = _fa()
     q, k, v, dO = inputs.for_workload(w)
     qd, kd, vd, dOd = (t.to(DEV) for t in (q, k, v, dO))
     o, lse = fa.fwd(qd, kd, vd, causal=w.causal)
     dq, dk, dv = fa.bwd(qd, kd, vd, o, dOd, lse, causal=w.causal)
+    out = tuple(t.cpu() for t in (o, lse, dq, dk, dv))
+    if grad_f32:
+        g32 = fa.bwd(qd, kd, vd, o, dOd, lse, causal=w.causal, grad_dtype=torch.float32)
+        out = out + tuple(t.cpu() for t in g32)
     fa.check_device_errors()
-    return (q, k, v, dO), tuple(t.cpu() for t in (o, lse, dq, dk, dv))
+    return (q, k, v, dO), out
 
 
-def _check_heads(w, cpu_in, gpu_out, heads, scaled=False):
+def _check_heads(w, cpu_in, gpu_out, heads):
+    """Whole heads against the oracle: O and lse at the absolute bounds; the
+    fp32-output gradients at the absolute 2e-2; the bf16-output gradients at
+    2e-2 plus bf16's own rounding of the result (assert_close_bf16_out)."""
     q, k, v, dO = cpu_in
-    o, lse, dq, dk, dv = gpu_out
-    cmp = assert_close_scaled if scaled else assert_close
+    o, lse, dq, dk, dv, dq32, dk32, dv32 = gpu_out
     for (b, h) in heads:
         sl = lambda t: t[b:b + 1, h:h + 1]
         o_r, lse_r = oracle.fwd(sl(q), sl(k), sl(v), causal=w.causal)
         dq_r, dk_r, dv_r, _, _ = oracle.bwd(sl(q), sl(k), sl(v), sl(dO), causal=w.causal)
         ctx = f"{w.name} head ({b},{h})"
-        cmp("o", sl(o), o_r, ctx=ctx)
+        assert_close("o", sl(o), o_r, ctx=ctx)
         assert_close("lse", sl(lse), lse_r, ctx=ctx)
-        cmp("dq", sl(dq), dq_r, ctx=ctx)
-        cmp("dk", sl(dk), dk_r, ctx=ctx)
-        cmp("dv", sl(dv), dv_r, ctx=ctx)
+        for name, g32, g16, r in (("dq", dq32, dq, dq_r), ("dk", dk32, dk, dk_r),
+                                  ("dv", dv32, dv, dv_r)):
+            assert_close(name, sl(g32), r, ctx=ctx + " fp32 out")
+            assert_close_bf16_out(name, sl(g16), r, ctx=ctx + " bf16 out")
 
 
 def _check_all_heads_properties(w, cpu_in, gpu_out):
@@ -81,21 +92,51 @@ def _check_all_heads_properties(w, cpu_in, gpu_out):
 
 
 def test_gpt_causal_workload():
-    """B=2, H=32, N=4096, d=128, causal: the benchmark workload."""
+    """B=2, H=32, N=4096, d=128, causal: the benchmark workload, 8 heads of
+    both batch entries against the oracle."""
     w = inputs.GPT_CAUSAL
-    cpu_in, gpu_out = _run(w)
-    _check_all_heads_properties(w, cpu_in, gpu_out)
-    _check_heads(w, cpu_in, gpu_out, [(0, 0), (1, 31), (0, 17)])
+    cpu_in, gpu_out = _run(w, grad_f32=True)
+    _check_all_heads_properties(w, cpu_in, gpu_out[:5])
+    _check_heads(w, cpu_in, gpu_out,
+                 [(0, 0), (0, 7), (0, 17), (0, 31), (1, 0), (1, 12), (1, 24), (1, 31)])
+
+
+LONG_CONTEXT_HEADS = [(0, 0), (0, 5), (0, 10), (0, 15)]
 
 
 def test_long_context_workload():
     """B=1, H=16, N=16384, d=128, causal, Q,K ~ N(0,3) with 1% of rows x8.
-    Logits reach the hundreds and gradients are far from unit scale, so the
-    bound on O and the gradients is scaled by the result's magnitude."""
+
+    O is a convex combination of V rows (|v| <= about 5), so the absolute
+    2e-2 bound applies to it whatever the logits, and so does lse's 1e-3.
+    The gradients are far from unit scale here (logits in the hundreds,
+    max|dQ| about 110): even with fp32 outputs their absolute errors are
+    0.59-0.65 (dQ), 0.18-0.36 (dK) and 0.031-0.039 (dV) on these four heads,
+    all above 2e-2, so the gradients alone are bounded by 2e-2 * max(1,
+    max|ref|) (normalised errors measured: at most 5.9e-3, 1.93e-2, 6.0e-4).
+    Both errors are recorded per head and tensor (FA_PARITY_RECORD)."""
     w = inputs.LONG_CONTEXT
-    cpu_in, gpu_out = _run(w)
-    _check_all_heads_properties(w, cpu_in, gpu_out)
-    _check_heads(w, cpu_in, gpu_out, [(0, 5)], scaled=True)
+    cpu_in, gpu_out = _run(w, grad_f32=True)
+    _check_all_heads_properties(w, cpu_in, gpu_out[:5])
+    q, k, v, dO = cpu_in
+    o, lse = gpu_out[0], gpu_out[1]
+    dq32, dk32, dv32 = gpu_out[5:]
+    for (b, h) in LONG_CONTEXT_HEADS:
+        sl = lambda t: t[b:b + 1, h:h + 1]
+        o_r, lse_r = oracle.fwd(sl(q), sl(k), sl(v), causal=w.causal)
+        dq_r, dk_r, dv_r, _, _ = oracle.bwd(sl(q), sl(k), sl(v), sl(dO), causal=w.causal)
+        ctx = f"{w.name} head ({b},{h})"
+        errs = {"o": assert_close("o", sl(o), o_r, ctx=ctx),
+                "lse": assert_close("lse", sl(lse), lse_r, ctx=ctx)}
+        for gd, grads in (("fp32", (dq32, dk32, dv32)), ("bf16", gpu_out[2:5])):
+            for name, a, r in zip(("dq", "dk", "dv"), grads, (dq_r, dk_r, dv_r)):
+                e = max_abs(sl(a), r)
+                mag = max(1.0, float(np.abs(r).max()))
+                record(workload=w.name, head=[b, h], tensor=name, grad_dtype=gd,
+                       abs_err=e, max_ref=mag, norm_err=e / mag)
+                errs[f"{name}_{gd}"] = e
+                assert e <= 2e-2 * mag, f"{name} ({gd}): {e:.3e} > 2e-2 * {mag:.3e} {ctx}"
+        record(workload=w.name, head=[b, h], errors=errs)
 
 
 @pytest.mark.parametrize("w", [inputs.MID_NC, inputs.MID_C], ids=lambda w: w.name)
@@ -116,8 +157,19 @@ def test_mid_workloads_every_head(w):
 def test_boundary_wave_sweep(w):
     """H=16, d in {64,128}, B in {1,8}, N in {1792,1793,2048,2049,4000,8192},
     both masks, forward and backward: ragged tails, masking and wave counts
-    on 148 SMs.  One head is checked against the oracle (the last head, whose
-    rows sit at the end of every buffer), all heads for properties."""
-    cpu_in, gpu_out = _run(w)
-    _check_all_heads_properties(w, cpu_in, gpu_out)
-    _check_heads(w, cpu_in, gpu_out, [(w.B - 1, w.H - 1)])
+    on 148 SMs.  Whole heads are checked against the oracle (sweep_heads),
+    all heads for properties."""
+    cpu_in, gpu_out = _run(w, grad_f32=True)
+    _check_all_heads_properties(w, cpu_in, gpu_out[:5])
+    _check_heads(w, cpu_in, gpu_out, sweep_heads(w))
+
+
+def sweep_heads(w):
+    """The heads of a sweep case checked against the oracle: every head when
+    B = 1, else a seeded subset of 4 that always includes the last one (whose
+    rows sit at the end of every buffer)."""
+    if w.B == 1:
+        return [(0, h) for h in range(w.H)]
+    rng = random.Random(f"{w.name}")
+    picks = rng.sample(range(w.B * w.H - 1), 3) + [w.B * w.H - 1]
+    return [divmod(i, w.H) for i in sorted(picks)]

@@ -38,11 +38,13 @@ def test_noalloc_rejects_oversized_problem_before_launch():
 @pytest.mark.gpu
 @pytest.mark.parametrize("causal", [False, True])
 def test_noalloc_matches_workspace_backward_twice(causal):
-    """Two calls in a row through the C ABI, each compared with fa_bwd on the
-    same inputs; the second call must not see the first call's scratch."""
+    """Calls in a row through the C ABI, each compared with fa_bwd on the same
+    inputs; no call may see an earlier call's scratch.  The third call
+    repeats the first shape, so its counters sit exactly where the first
+    call left its own: a counter that was not cleared would change it."""
     fa, _ = _lib()
     dev = "cuda:0"
-    for call, (B, H, N, d) in enumerate([(1, 3, 300, 128), (2, 2, 777, 64)]):
+    for call, (B, H, N, d) in enumerate([(1, 3, 300, 128), (2, 2, 777, 64), (1, 3, 300, 128)]):
         q, k, v, dO = (t.to(dev) for t in inputs.qkv_do(B, H, N, d, seed=40 + call))
         o, lse = fa.fwd(q, k, v, causal=causal)
         ref = fa.bwd(q, k, v, o, dO, lse, causal=causal)

@@ -42,6 +42,8 @@
 // for the two pipeline slots s; dQ^T of slot s overwrites dP^T_s once the
 // compute warps have read it, P^T_s (bf16 pairs) overwrites S^T_s.
 #pragma once
+#include <cfloat>
+
 #include "sm100.cuh"
 
 namespace fa {
@@ -531,6 +533,36 @@ __device__ void bwd_compute(const BwdParams& p, uint8_t* smem, BwdBarriers* b, u
 // shared memory (32 rows at a time, two buffers) and adds it into the fp32
 // accumulator with bulk reduce-add copies, one in flight while the other
 // buffer fills.
+//
+// The 128 drain threads meet at named barriers, so they must agree on every
+// wait's outcome: each wait ends with a barrier reduction over the 128
+// threads, and on an abort all four warps leave together (none is left
+// waiting at a named barrier for a warp that has gone).
+
+// True on every drain thread iff `ok` holds on all 128 (barrier 1).
+__device__ __forceinline__ bool drain_all(bool ok) {
+  uint32_t r;
+  asm volatile(
+      "{\n\t.reg .pred p, q;\n\t"
+      "setp.ne.u32 p, %1, 0;\n\t"
+      "bar.red.and.pred q, 1, 128, p;\n\t"
+      "selp.u32 %0, 1, 0, q;\n\t}\n"
+      : "=r"(r)
+      : "r"(static_cast<uint32_t>(ok))
+      : "memory");
+  return r != 0;
+}
+
+// A bounded mbarrier wait by every drain thread, with one answer for all.
+__device__ __forceinline__ bool drain_wait(uint64_t* bar, uint32_t parity, BwdBarriers* b,
+                                           int* status) {
+  bool ok = !*(volatile int*)&b->abort_flag;
+  if (ok) ok = mbar_wait(bar, parity, status);
+  ok = drain_all(ok);
+  if (!ok) *(volatile int*)&b->abort_flag = 1;
+  return ok;
+}
+
 template <int D, bool CAUSAL>
 __device__ void bwd_drain(const BwdParams& p, uint8_t* smem, BwdBarriers* b, uint32_t tmem) {
   using L = BwdLayout<D>;
@@ -544,16 +576,23 @@ __device__ void bwd_drain(const BwdParams& p, uint8_t* smem, BwdBarriers* b, uin
   const bool issuer = (t == 0);
   int g = 0, rc = 0;
   for (;;) {
-    const int w = next_unit_warp(b, rc, p.status);
+    // Next unit from the ring, with one answer for the four warps.
+    const int slot = rc % kUnitRing;
+    if (!drain_wait(&b->unit_full[slot], (rc / kUnitRing) & 1, b, p.status)) break;
+    const int w = *(volatile int*)&b->unit_id[slot];
+    __syncwarp();
+    if (lane_id() == 0) mbar_arrive(&b->unit_empty[slot]);
+    ++rc;
     if (w < 0) break;
     const BwdUnit u = bwd_decode<CAUSAL>(p, w);
+    bool ok = true;
     for (int it = 0; it < u.n; ++it, ++g) {
       const int s = g & 1;
       const int q0 = (u.i0 + it) * 64;
-      if (!bwait_warp(&b->dq_full[s], (g >> 1) & 1, b, p.status)) {
-        if (issuer) bulk_wait0();
-        return;
-      }
+      // Each warp waits and reads its TMEM quarter on its own; the four
+      // agree on the outcome at the barrier before the first staging write.
+      // (After a failed wait the values read are dropped there.)
+      ok = !*(volatile int*)&b->abort_flag && mbar_wait(&b->dq_full[s], (g >> 1) & 1, p.status);
       tc_fence_after();
       uint32_t r[64];
       tmem_ld_x64(tmem + lane_base + L::kTdP + 64 * s, r);
@@ -564,7 +603,15 @@ __device__ void bwd_drain(const BwdParams& p, uint8_t* smem, BwdBarriers* b, uin
       for (int half = 0; half < 2; ++half) {
         float* stage = reinterpret_cast<float*>(smem + L::kStage + half * L::kStageBytes);
         if (issuer) bulk_wait_read1();  // this buffer's previous reduce has read it
-        named_bar_sync(1, 128);
+        if (half == 0) {
+          ok = drain_all(ok);
+          if (!ok) {
+            *(volatile int*)&b->abort_flag = 1;
+            break;
+          }
+        } else {
+          named_bar_sync(1, 128);
+        }
         if (valid) {
 #pragma unroll
           for (int c = 0; c < L::kStageRows; ++c)
@@ -581,9 +628,11 @@ __device__ void bwd_drain(const BwdParams& p, uint8_t* smem, BwdBarriers* b, uin
           bulk_commit();  // an empty group keeps the two-buffer accounting exact
         }
       }
+      if (!ok) break;
     }
+    if (!ok) break;
   }
-  if (issuer) bulk_wait0();
+  if (issuer) bulk_wait0();  // no copy may read shared memory after the CTA exits
 }
 
 // ---------------------------------------------------------------- kernels
@@ -677,13 +726,14 @@ __global__ void __launch_bounds__(512, 1)
 }
 
 // D_i = rowsum(dO * O); lse2 = lse * log2(e) (+inf and D = 0 on rows N..Npad);
-// zero the dQ accumulator and the work-unit counter.  One thread per 8 consecutive elements of a row.
+// zero the dQ accumulator and the work-unit counter; latch the assert bit if
+// an lse is not finite.  One thread per 8 consecutive elements of a row.
 template <int D>
 __global__ void __launch_bounds__(256)
     fa_bwd_prep(const __nv_bfloat16* __restrict__ o, const __nv_bfloat16* __restrict__ dO,
                 const float* __restrict__ lse, float* __restrict__ lse2, float* __restrict__ dvec,
                 float* __restrict__ dq_acc, int* __restrict__ sched, int BH, int N, int Npad,
-                int zero_acc) {
+                int zero_acc, int* __restrict__ status) {
   constexpr int TPR = D / 8;  // threads per row
   if (blockIdx.x == 0 && threadIdx.x == 0) *sched = 0;
   const long long gid = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x;
@@ -717,8 +767,11 @@ __global__ void __launch_bounds__(256)
   for (int m = TPR / 2; m >= 1; m >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, m, TPR);
   if (in_range && part == 0) {
     const size_t i = static_cast<size_t>(bh) * Npad + q;
+    const float l = real ? lse[static_cast<size_t>(bh) * N + q] : 0.f;
+    // Consistency check: a forward's lse is finite on every row.
+    if (real && !(fabsf(l) <= FLT_MAX)) atomicOr(status, kDevAssert);
     dvec[i] = real ? acc : 0.f;
-    lse2[i] = real ? lse[static_cast<size_t>(bh) * N + q] * 1.4426950408889634f : INFINITY;
+    lse2[i] = real ? l * 1.4426950408889634f : INFINITY;
   }
 }
 

@@ -291,11 +291,11 @@ int launch_bwd(const void* q, const void* k, const void* v, const void* o, const
     if (d == 64)
       fa::fa_bwd_prep<64><<<blocks, 256, 0, stream>>>(
           static_cast<const __nv_bfloat16*>(o), static_cast<const __nv_bfloat16*>(dO), lse, lse2,
-          dvec, dq_acc, sched, BH, N, static_cast<int>(npad), deterministic ? 0 : 1);
+          dvec, dq_acc, sched, BH, N, static_cast<int>(npad), deterministic ? 0 : 1, status);
     else
       fa::fa_bwd_prep<128><<<blocks, 256, 0, stream>>>(
           static_cast<const __nv_bfloat16*>(o), static_cast<const __nv_bfloat16*>(dO), lse, lse2,
-          dvec, dq_acc, sched, BH, N, static_cast<int>(npad), deterministic ? 0 : 1);
+          dvec, dq_acc, sched, BH, N, static_cast<int>(npad), deterministic ? 0 : 1, status);
     if (cudaPeekAtLastError() != cudaSuccess) return FA_ERR_LAUNCH;
   }
   // 2. tensor-core main kernel

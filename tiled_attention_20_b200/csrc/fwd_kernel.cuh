@@ -590,6 +590,13 @@ __device__ void fwd_softmax(const FwdParams& p, FwdBarriers* b, uint32_t tmem, i
             pack_bf16x2(__uint_as_float(o[8 * v + 6]) * inv_l, __uint_as_float(o[8 * v + 7]) * inv_l));
     }
     if (valid) p.lse[static_cast<size_t>(u.bh) * N + row] = (m_used + __log2f(l)) * 0.69314718055994531f;
+    // Consistency check: the reference maximum never exceeds the row's
+    // maximum score, so that key alone adds 2^0 = 1 to the normaliser, up to
+    // the rounding of the exponent and of the exponential (relative 2^-13 at
+    // worst, also after E4M3 rounding of p); a normaliser below 1/2, or not
+    // finite (which non-finite inputs also give), latches the assert bit.
+    if (valid && !(((FP8 ? lq : l) >= 0.5f) && ((FP8 ? lq : l) <= FLT_MAX)))
+      atomicOr(p.status, kDevAssert);
   }
 }
 

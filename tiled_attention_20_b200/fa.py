@@ -32,7 +32,7 @@ EXPORTED = ["fa_fwd", "fa_bwd", "fa_bwd_workspace_size", "fa_strerror",
             "fa_gemm", "fa_gemm_workspace_size", "fa_gemm_tiles", "fa_selftest_wait_timeout",
             "fa_fwd_schedule"]
 NOALLOC_MAX_SCRATCH = 32 << 20  # FA_BWD_NOALLOC_MAX_SCRATCH
-KERNEL_IDS = {0: "fa_fwd_kernel", 1: "fa_bwd_prep", 2: "fa_bwd_kernel", 3: "fa_bwd_dq_convert",
+KERNEL_IDS = {0: "fa_fwd_kernel", 1: "fa_bwd_prep", 2: "fa_bwd_kernel", 3: "unused",
               4: "fa_dq_kernel", 5: "fa_decode_kernel", 6: "fa_gemm_kernel", 7: "fa_gemm_pack"}
 DECODE_MAX_NQ = 8
 
@@ -138,6 +138,24 @@ def _check_qkv(*ts):
             raise ValueError("inputs must be on one device")
 
 
+def _check_buffer(name, t, device, dtype, shape=None, min_numel=None):
+    """A tensor the caller passes for the library to read or write: on
+    `device`, of `dtype`, contiguous, and of `shape` (or at least `min_numel`
+    elements).  Raises ValueError before anything reaches libfa."""
+    if not torch.is_tensor(t):
+        raise ValueError(f"{name} must be a torch tensor")
+    if t.device != device:
+        raise ValueError(f"{name} must be on {device} (got {t.device})")
+    if t.dtype != dtype:
+        raise ValueError(f"{name} must be {dtype} (got {t.dtype})")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if shape is not None and tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} must have shape {tuple(shape)} (got {tuple(t.shape)})")
+    if min_numel is not None and t.numel() < min_numel:
+        raise ValueError(f"{name} needs at least {min_numel} elements (got {t.numel()})")
+
+
 def default_scale(d: int) -> float:
     return 1.0 / math.sqrt(d)
 
@@ -151,6 +169,8 @@ def fwd(q, k, v, scale=None, causal=False, out=None, lse=None):
         out = torch.empty_like(q)
     if lse is None:
         lse = torch.empty((B, H, N), dtype=torch.float32, device=q.device)
+    _check_buffer("out", out, q.device, torch.bfloat16, q.shape)
+    _check_buffer("lse", lse, q.device, torch.float32, (B, H, N))
     with torch.cuda.device(q.device):
         st = load().fa_fwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(),
                            lse.data_ptr(), B, H, N, d, scale, int(bool(causal)), _stream(q.device))
@@ -180,6 +200,8 @@ def fwd_fp8(q, k, v, descale_q, descale_k, descale_v, scale=None, causal=False, 
         out = torch.empty(q.shape, dtype=torch.bfloat16, device=q.device)
     if lse is None:
         lse = torch.empty((B, H, N), dtype=torch.float32, device=q.device)
+    _check_buffer("out", out, q.device, torch.bfloat16, q.shape)
+    _check_buffer("lse", lse, q.device, torch.float32, (B, H, N))
     with torch.cuda.device(q.device):
         st = load().fa_fwd_fp8(q.data_ptr(), k.data_ptr(), v.data_ptr(), descale_q.data_ptr(),
                                descale_k.data_ptr(), descale_v.data_ptr(), out.data_ptr(),
@@ -193,22 +215,38 @@ def workspace_size(B, H, N, d) -> int:
     return int(load().fa_bwd_workspace_size(B, H, N, d))
 
 
+def _grad_code(grad_dtype) -> int:
+    codes = {torch.bfloat16: 0, torch.float32: 1}
+    if grad_dtype not in codes:
+        raise ValueError("grad_dtype must be torch.bfloat16 or torch.float32")
+    return codes[grad_dtype]
+
+
+def _grad_buffers(q, grad_dtype, dq, dk, dv):
+    """dq, dk, dv as given (checked) or freshly allocated."""
+    out = []
+    for name, t in (("dq", dq), ("dk", dk), ("dv", dv)):
+        if t is None:
+            t = torch.empty(q.shape, dtype=grad_dtype, device=q.device)
+        _check_buffer(name, t, q.device, grad_dtype, q.shape)
+        out.append(t)
+    return out
+
+
 def bwd(q, k, v, o, dO, lse, scale=None, causal=False, grad_dtype=torch.bfloat16,
         workspace=None, dq=None, dk=None, dv=None, deterministic=False):
     """dQ, dK, dV [B,H,N,d] (bf16 or fp32) for the forward that produced o, lse.
     deterministic=True calls fa_bwd_deterministic (bit-reproducible dQ)."""
     _check_qkv(q, k, v, o, dO)
     B, H, N, d = q.shape
-    if lse.dtype != torch.float32 or tuple(lse.shape) != (B, H, N) or not lse.is_contiguous():
-        raise ValueError("lse must be contiguous fp32 [B, H, N]")
+    _check_buffer("lse", lse, q.device, torch.float32, (B, H, N))
     scale = default_scale(d) if scale is None else float(scale)
-    gd = {torch.bfloat16: 0, torch.float32: 1}[grad_dtype]
+    gd = _grad_code(grad_dtype)
     ws_bytes = workspace_size(B, H, N, d)
     if workspace is None:
         workspace = torch.empty(max(ws_bytes, 16), dtype=torch.uint8, device=q.device)
-    dq = torch.empty(q.shape, dtype=grad_dtype, device=q.device) if dq is None else dq
-    dk = torch.empty(q.shape, dtype=grad_dtype, device=q.device) if dk is None else dk
-    dv = torch.empty(q.shape, dtype=grad_dtype, device=q.device) if dv is None else dv
+    _check_buffer("workspace", workspace, q.device, torch.uint8, min_numel=ws_bytes)
+    dq, dk, dv = _grad_buffers(q, grad_dtype, dq, dk, dv)
     with torch.cuda.device(q.device):
         fn = load().fa_bwd_deterministic if deterministic else load().fa_bwd
         st = fn(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(),
@@ -229,13 +267,10 @@ def bwd_noalloc(q, k, v, o, dO, lse, scale=None, causal=False, grad_dtype=torch.
     that overlap on the GPU share the scratch and must not run concurrently."""
     _check_qkv(q, k, v, o, dO)
     B, H, N, d = q.shape
-    if lse.dtype != torch.float32 or tuple(lse.shape) != (B, H, N) or not lse.is_contiguous():
-        raise ValueError("lse must be contiguous fp32 [B, H, N]")
+    _check_buffer("lse", lse, q.device, torch.float32, (B, H, N))
     scale = default_scale(d) if scale is None else float(scale)
-    gd = {torch.bfloat16: 0, torch.float32: 1}[grad_dtype]
-    dq = torch.empty(q.shape, dtype=grad_dtype, device=q.device) if dq is None else dq
-    dk = torch.empty(q.shape, dtype=grad_dtype, device=q.device) if dk is None else dk
-    dv = torch.empty(q.shape, dtype=grad_dtype, device=q.device) if dv is None else dv
+    gd = _grad_code(grad_dtype)
+    dq, dk, dv = _grad_buffers(q, grad_dtype, dq, dk, dv)
     with torch.cuda.device(q.device):
         st = load().fa_bwd_noalloc(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(),
                                    dO.data_ptr(), lse.data_ptr(), dq.data_ptr(), dk.data_ptr(),
