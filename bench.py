@@ -54,6 +54,8 @@ import torch  # noqa: E402
 from tiled_attention_20_b200 import inputs, perf, ranks  # noqa: E402
 
 WORKLOAD = inputs.GPT_CAUSAL
+ATTN_WORKLOADS = {w.name: w for w in (inputs.SMALL_FWD, inputs.MID_NC, inputs.MID_C,
+                                      inputs.GPT_CAUSAL, inputs.LONG_CONTEXT)}
 DECODE_WORKLOADS = {w.name: w for w in (inputs.DECODE_B8, inputs.DECODE_B8_RAGGED,
                                         inputs.DECODE_SPEC, inputs.DECODE_LONG)}
 METRIC = "attention fwd+bwd TFLOP/s (bf16, causal, N=4096 d=128) and % of dense BF16 peak"
@@ -89,21 +91,44 @@ def parse_args():
     ap.add_argument("--decode", default=None, metavar="WORKLOAD",
                     choices=sorted(DECODE_WORKLOADS),
                     help="time fa_decode on one decode workload instead of fwd+bwd")
+    ap.add_argument("--workload", default=WORKLOAD.name, choices=sorted(ATTN_WORKLOADS),
+                    help="attention workload of the fwd+bwd step (default: the benchmark's)")
+    ap.add_argument("--quick", action="store_true",
+                    help="headline pass only (no distribution or trace pass): for profiler runs")
+    ap.add_argument("--sweep", action="store_true",
+                    help="time forward and backward of the 48-case boundary/wave sweep instead")
+    ap.add_argument("--cpu-table", action="store_true",
+                    help="time the fp64 oracle on the small, mid and GPT-style workloads "
+                         "(fwd and fwd+bwd; the small one also on one thread) instead")
     return ap.parse_args()
 
 
 def workload_config(w=WORKLOAD, extra=None):
+    in_bytes = 4 * w.B * w.H * w.N * w.d * 2  # Q, K, V, dO
     cfg = {"workload": w.name, "B": w.B, "H": w.H, "N": w.N, "d": w.d, "causal": w.causal,
-           "passes": "fwd+bwd", "dist": w.dist, "seed": w.seed,
-           "l2": "inputs_exceed_l2 (no flush)"}
+           "passes": "fwd+bwd" if w.backward else "fwd", "dist": w.dist, "seed": w.seed,
+           "l2": ("inputs_exceed_l2 (no flush)" if in_bytes > 126e6 else
+                  "inputs_fit_l2 (no flush: compute-bound)")}
     if extra:
         cfg.update(extra)
     return cfg
 
 
+def workload_metric(w) -> str:
+    """The headline metric for the benchmark workload; the same measure,
+    named by its shape, for the others."""
+    if w == WORKLOAD:
+        return METRIC
+    mask = "causal" if w.causal else "non-causal"
+    return (f"attention {'fwd+bwd' if w.backward else 'fwd'} TFLOP/s (bf16, {mask}, "
+            f"B={w.B} H={w.H} N={w.N} d={w.d}) and % of dense BF16 peak")
+
+
 def step_flops(w=WORKLOAD) -> float:
-    return (perf.attention_flops(w.B, w.H, w.N, w.d, w.causal, False) +
-            perf.attention_flops(w.B, w.H, w.N, w.d, w.causal, True))
+    f = perf.attention_flops(w.B, w.H, w.N, w.d, w.causal, False)
+    if w.backward:
+        f += perf.attention_flops(w.B, w.H, w.N, w.d, w.causal, True)
+    return f
 
 
 def measured_peaks():
@@ -241,17 +266,17 @@ class ClockSampler:
 
 
 # ---------------------------------------------------------------- timing
-def timed_passes(step, steps, stream, dev, dist, world):
-    """Three timed passes of `step` on `stream`, each bracketed by a barrier
+def timed_passes(step, steps, stream, dev, dist, world, quick=False):
+    """Two timed passes of `step` on `stream`, each bracketed by a barrier
     and a synchronize:
-      1. the headline: `steps` steps back to back between two CUDA events,
-         nothing else on the stream (so consecutive kernels may overlap their
-         boundaries); returns the mean step time, max over ranks;
+      1. the headline: `steps` steps between two CUDA events, with every
+         library launch also bracketed by events (fa.trace_start/stop), so
+         the per-kernel times come from the timed region itself; returns the
+         mean step time, max over ranks;
       2. the distribution: max(100, steps) steps with an event after each,
-         for the median, 10th and 90th percentile of the step time;
-      3. the per-kernel trace: `steps` steps with every library launch
-         bracketed by events (fa.trace_start / trace_stop).
-    Returns (mean ms, stats dict, traced kernels)."""
+         for the median, 10th and 90th percentile of the step time.
+    With quick (profiler runs), pass 1 runs without the trace and pass 2 is
+    skipped.  Returns (mean ms, stats dict, traced kernels)."""
     import tiled_attention_20_b200.fa as fa
 
     def sync():
@@ -262,12 +287,17 @@ def timed_passes(step, steps, stream, dev, dist, world):
     sync()
     e0 = torch.cuda.Event(enable_timing=True)
     e1 = torch.cuda.Event(enable_timing=True)
+    if not quick:
+        fa.trace_start()
     e0.record(stream)
     for _ in range(steps):
         step()
     e1.record(stream)
     sync()
+    traced = {} if quick else fa.trace_stop()
     ms = ranks.max_over_ranks(e0.elapsed_time(e1) / steps, dist, dev)
+    if quick:
+        return ms, {}, traced
 
     n = max(100, steps)
     ev = [torch.cuda.Event(enable_timing=True) for _ in range(n + 1)]
@@ -279,21 +309,18 @@ def timed_passes(step, steps, stream, dev, dist, world):
     per = sorted(ev[i].elapsed_time(ev[i + 1]) for i in range(n))
     pick = lambda f: per[min(n - 1, int(round(f * (n - 1))))]
     stats = {"n": n, "median_ms": statistics.median(per), "p10_ms": pick(0.1),
-             "p90_ms": pick(0.9), "min_ms": per[0], "max_ms": per[-1]}
-
-    fa.trace_start()
-    for _ in range(steps):
-        step()
-    sync()
-    traced = fa.trace_stop()
+             "p90_ms": pick(0.9), "min_ms": per[0], "max_ms": per[-1],
+             "after": "the headline pass (its clock may be lower: power cap)"}
     return ms, stats, traced
 
 
 # ---------------------------------------------------------------- CPU oracle
-def cpu_oracle_rate(q, k, v, dO, w, seconds: float):
+def cpu_oracle_rate(q, k, v, dO, w, seconds: float, backward=None):
     """The oracle (fp64, as it stands) on whole heads of the workload until
-    `seconds` of wall time have passed; returns (TFLOP/s, heads, cores, s)."""
+    `seconds` of wall time have passed (forward, and backward when the
+    workload has one); returns (TFLOP/s, heads, cores, s)."""
     import oracle  # the benchmark's CPU-baseline leg is one of the oracle's permitted users
+    backward = w.backward if backward is None else backward
     t0 = time.time()
     heads = 0
     total = w.B * w.H
@@ -301,14 +328,124 @@ def cpu_oracle_rate(q, k, v, dO, w, seconds: float):
         b, h = divmod(heads, w.H)
         sl = lambda t: t[b:b + 1, h:h + 1]
         oracle.fwd(sl(q), sl(k), sl(v), causal=w.causal)
-        oracle.bwd(sl(q), sl(k), sl(v), sl(dO), causal=w.causal)
+        if backward:
+            oracle.bwd(sl(q), sl(k), sl(v), sl(dO), causal=w.causal)
         heads += 1
         if time.time() - t0 >= seconds:
             break
     el = time.time() - t0
-    fl = (perf.attention_flops(1, 1, w.N, w.d, w.causal, False) +
-          perf.attention_flops(1, 1, w.N, w.d, w.causal, True)) * heads
-    return fl / el / 1e12, heads, oracle.num_threads(), el
+    fl = perf.attention_flops(1, 1, w.N, w.d, w.causal, False)
+    if backward:
+        fl += perf.attention_flops(1, 1, w.N, w.d, w.causal, True)
+    return fl * heads / el / 1e12, heads, oracle.num_threads(), el
+
+
+def cpu_model() -> str:
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    return "unknown"
+
+
+def run_cpu_table(args):
+    """The fp64 oracle, as it stands, on the host cores: forward and
+    forward+backward wall time of whole workloads (small, both mid masks,
+    GPT-style), the small one also on one thread.  One JSON line."""
+    import oracle
+    rows = []
+    for w in (inputs.SMALL_FWD, inputs.MID_NC, inputs.MID_C, inputs.GPT_CAUSAL):
+        q, k, v, dO = inputs.for_workload(w)
+        for backward in ((False,) if not w.backward else (False, True)):
+            for threads in ((0, 1) if w is inputs.SMALL_FWD else (0,)):
+                all_cores = oracle.num_threads()
+                if threads:
+                    oracle.set_num_threads(threads)
+                rate, heads, cores, el = cpu_oracle_rate(q, k, v, dO, w, float("inf"), backward)
+                oracle.set_num_threads(all_cores)
+                rows.append({"workload": w.name, "passes": "fwd+bwd" if backward else "fwd",
+                             "threads": cores, "heads": heads, "seconds": el,
+                             "gflops": rate * 1e3})
+    print(json.dumps({"metric": "fp64 CPU oracle wall time (whole workloads)",
+                      "cpu_model": cpu_model(), "nproc": os.cpu_count(), "rows": rows}),
+          flush=True)
+
+
+SWEEP_METRIC = "attention TFLOP/s vs N, boundary/wave sweep (bf16, H=16)"
+
+
+def run_sweep(args, rank, world, local_rank, dist):
+    """Forward and backward of each of the 48 sweep workloads, timed with
+    CUDA events (mean of `reps` launches each after warm-up), with the work
+    units and waves of 148 SMs beside the rate.  Rank 0 prints one JSON line
+    whose value is the median fwd+bwd rate over the cases."""
+    import tiled_attention_20_b200.fa as fa
+    from tiled_attention_20_b200 import build as fa_build
+    if rank == 0 or world == 1:
+        fa_build.build()
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    sms = torch.cuda.get_device_properties(dev).multi_processor_count
+    stream = torch.cuda.current_stream(dev)
+    peaks, peaks_src = measured_peaks()
+    reps = max(5, min(args.steps, 50))
+    sampler = ClockSampler(dev.index if world == 1 else local_rank)
+    sampler.start()
+    time.sleep(0.4)
+    rows = []
+    launches = 0
+    for w in inputs.sweep_workloads():
+        q, k, v, dO = (t.to(dev) for t in inputs.for_workload(w))
+        o = torch.empty_like(q)
+        lse = torch.empty((w.B, w.H, w.N), dtype=torch.float32, device=dev)
+        grads = [torch.empty_like(q) for _ in range(3)]
+        ws = torch.empty(fa.workspace_size(w.B, w.H, w.N, w.d), dtype=torch.uint8, device=dev)
+
+        def timed(fn):
+            for _ in range(3):
+                fn()
+            e0 = torch.cuda.Event(enable_timing=True)
+            e1 = torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            for _ in range(reps):
+                fn()
+            e1.record(stream)
+            e1.synchronize()
+            return e0.elapsed_time(e1) / reps
+
+        fwd = lambda: fa.fwd(q, k, v, causal=w.causal, out=o, lse=lse)
+        bwd = lambda: fa.bwd(q, k, v, o, dO, lse, causal=w.causal, workspace=ws, dq=grads[0],
+                             dk=grads[1], dv=grads[2])
+        ms_f = timed(fwd)
+        ms_b = timed(bwd)
+        launches += (3 + reps) * 4  # forward + preprocess, main, conversion
+        f_f = perf.attention_flops(w.B, w.H, w.N, w.d, w.causal, False)
+        f_b = perf.attention_flops(w.B, w.H, w.N, w.d, w.causal, True)
+        ctas_f, units_f = fa.launch_shape(0, w.B, w.H, w.N, w.d, w.causal)
+        ctas_b, units_b = fa.launch_shape(1, w.B, w.H, w.N, w.d, w.causal)
+        rows.append({"workload": w.name, "N": w.N, "d": w.d, "B": w.B, "causal": w.causal,
+                     "fwd_ms": ms_f, "bwd_ms": ms_b, "fwd_tflops": f_f / ms_f / 1e9,
+                     "bwd_tflops": f_b / ms_b / 1e9,
+                     "fwdbwd_tflops": (f_f + f_b) / (ms_f + ms_b) / 1e9,
+                     "fwd_units": units_f, "bwd_units": units_b,
+                     "fwd_waves": units_f / sms, "bwd_waves": units_b / sms})
+        del q, k, v, dO, o, lse, grads, ws
+    clocks = sampler.stop()
+    fa.check_device_errors(dev)
+    if rank == 0:
+        rates = sorted(r["fwdbwd_tflops"] for r in rows)
+        value = statistics.median(rates)
+        print(json.dumps({
+            "metric": SWEEP_METRIC, "value": value, "unit": UNIT, "n_gpus": world,
+            "steps": reps, "warmup": 3, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": {"workload": "boundary_wave_sweep_48", "value": "median fwd+bwd over cases",
+                       "l2": "no flush (compute-bound)", "sms": sms},
+            "pct_of_peak": value / peaks["bf16_tflops"], "peak_source": peaks_src,
+            "gpu_launches": launches, "clocks": clocks, "sweep": rows}), flush=True)
 
 
 def run_reference(args, rank, world):
@@ -365,7 +502,7 @@ def run_ours(args, rank, world, local_rank, dist):
         dist.barrier()
     dev = torch.device("cuda", local_rank)
     torch.cuda.set_device(dev)
-    w = WORKLOAD
+    w = ATTN_WORKLOADS[args.workload]
     q_h, k_h, v_h, dO_h = inputs.qkv_do(w.B, w.H, w.N, w.d, seed=ranks.rank_seed(w.seed, rank),
                                         dist=w.dist)
     q, k, v, dO = (t.to(dev) for t in (q_h, k_h, v_h, dO_h))
@@ -376,14 +513,15 @@ def run_ours(args, rank, world, local_rank, dist):
 
     def step():
         fa.fwd(q, k, v, causal=w.causal, out=o, lse=lse)
-        fa.bwd(q, k, v, o, dO, lse, causal=w.causal, workspace=ws, dq=dq, dk=dk, dv=dv,
-               deterministic=args.deterministic)
+        if w.backward:
+            fa.bwd(q, k, v, o, dO, lse, causal=w.causal, workspace=ws, dq=dq, dk=dk, dv=dv,
+                   deterministic=args.deterministic)
 
     # Output check before timing (no oracle here): finite results, and row 0
     # of a causal head sees only key 0, so O_0 must equal V_0 bit for bit.
     step()
     fa.check_device_errors(dev)
-    for t in (o, lse, dq, dk, dv):
+    for t in (o, lse, dq, dk, dv) if w.backward else (o, lse):
         if not torch.isfinite(t).all():
             raise RuntimeError("non-finite output")
     if w.causal and not torch.equal(o[:, :, 0], v[:, :, 0]):
@@ -398,11 +536,17 @@ def run_ours(args, rank, world, local_rank, dist):
     # keep the GPU busy while the sampler starts, outside the timed region
     for _ in range(max(3, args.warmup)):
         step()
-    ms, stats, traced = timed_passes(step, args.steps, stream, dev, dist, world)
+    ms, stats, traced = timed_passes(step, args.steps, stream, dev, dist, world, args.quick)
     clocks = sampler.stop()
     fa.check_device_errors(dev)
     flops = step_flops(w)
     value = ranks.weak_scaling_rate(flops, world, ms) / 1e12
+    if args.quick:  # a profiler run: the headline pass alone
+        if rank == 0:
+            print(json.dumps({"metric": workload_metric(w), "value": value, "unit": UNIT,
+                              "ms_per_step": ms, "config": workload_config(w), "quick": True}),
+                  flush=True)
+        return
     stats["tflops_at_median"] = flops / (stats["median_ms"] * 1e-3) / 1e12
 
     # dominant kernel by traced time
@@ -438,17 +582,22 @@ def run_ours(args, rank, world, local_rank, dist):
     # end to end through the public API with host buffers
     e2e = None
     if not args.no_e2e:
-        host_in = [t.pin_memory() for t in (q_h, k_h, v_h, dO_h)]
-        host_out = [torch.empty(t.shape, dtype=t.dtype).pin_memory() for t in (o, lse, dq, dk, dv)]
-        dev_in = [[q, k, v, dO], [torch.empty_like(t) for t in (q, k, v, dO)]]
-        dev_out = [[o, lse, dq, dk, dv], [torch.empty_like(t) for t in (o, lse, dq, dk, dv)]]
+        ins = (q_h, k_h, v_h, dO_h) if w.backward else (q_h, k_h, v_h)
+        outs = (o, lse, dq, dk, dv) if w.backward else (o, lse)
+        host_in = [t.pin_memory() for t in ins]
+        host_out = [torch.empty(t.shape, dtype=t.dtype).pin_memory() for t in outs]
+        dev_in = [[t.to(dev) for t in ins], [torch.empty(t.shape, dtype=t.dtype, device=dev)
+                                             for t in ins]]
+        dev_out = [list(outs), [torch.empty_like(t) for t in outs]]
 
         def run(kset):
-            qq, kk, vv, dd = dev_in[kset]
-            oo, ll, gq, gk, gv = dev_out[kset]
+            qq, kk, vv = dev_in[kset][:3]
+            oo, ll = dev_out[kset][:2]
             fa.fwd(qq, kk, vv, causal=w.causal, out=oo, lse=ll)
-            fa.bwd(qq, kk, vv, oo, dd, ll, causal=w.causal, workspace=ws, dq=gq, dk=gk, dv=gv,
-                   deterministic=args.deterministic)
+            if w.backward:
+                gq, gk, gv = dev_out[kset][2:]
+                fa.bwd(qq, kk, vv, oo, dev_in[kset][3], ll, causal=w.causal, workspace=ws,
+                       dq=gq, dk=gk, dv=gv, deterministic=args.deterministic)
 
         n_e2e = max(1, args.e2e_steps)
         ms_e2e = ranks.max_over_ranks(
@@ -470,7 +619,7 @@ def run_ours(args, rank, world, local_rank, dist):
 
     if rank == 0:
         line = {
-            "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
+            "metric": workload_metric(w), "value": value, "unit": UNIT, "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
             "dtype": "bf16", "data": "synthetic",
@@ -901,6 +1050,10 @@ def main():
     if args.impl == "reference":
         run_reference(args, rank, world)
         return
+    if args.cpu_table:
+        if rank == 0:
+            run_cpu_table(args)
+        return
     dist = None
     if world > 1:
         import datetime
@@ -914,6 +1067,8 @@ def main():
             run_fp8(args, rank, world, local_rank, dist)
         elif args.gemm_sweep:
             run_gemm_sweep(args, rank, world, local_rank, dist)
+        elif args.sweep:
+            run_sweep(args, rank, world, local_rank, dist)
         else:
             run_ours(args, rank, world, local_rank, dist)
     finally:
