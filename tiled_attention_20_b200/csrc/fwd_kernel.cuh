@@ -107,14 +107,16 @@ struct FwdUnit {
 };
 
 // One Q tile pair of one head: its first row and the key tiles each of its
-// two Q tiles reads (all of them, or up to the diagonal when causal).
+// two Q tiles reads (all of them, or up to the diagonal when causal).  A
+// second tile that lies wholly past the last row (N mod 256 in [1, 128])
+// reads none: it holds no query.
 __device__ __forceinline__ FwdUnit fwd_pair(const FwdParams& p, int bh, int qt2, bool causal) {
   FwdUnit u;
   u.bh = bh;
   u.q0 = qt2 * 256;
   const int nkv = (p.N + 127) / 128;
   u.nk0 = causal ? min(2 * qt2 + 1, nkv) : nkv;
-  u.nk1 = causal ? min(2 * qt2 + 2, nkv) : nkv;
+  u.nk1 = (u.q0 + 128 >= p.N) ? 0 : (causal ? min(2 * qt2 + 2, nkv) : nkv);
   return u;
 }
 
@@ -226,7 +228,7 @@ __device__ void fwd_producer(const CUtensorMap* tm_q, const CUtensorMap* tm_k,
       tma_load_3d(smem + L::kQ0 + c * 16384, tm_q, &b->q_full, c * 64, u.q0, u.bh);
       tma_load_3d(smem + L::kQ1 + c * 16384, tm_q, &b->q_full, c * 64, u.q0 + 128, u.bh);
     }
-    const int nk = u.nk1;
+    const int nk = max(u.nk0, u.nk1);
     for (int j = 0; j < nk; ++j) {
       {
         const int st = kc % S;
@@ -328,7 +330,7 @@ __device__ void fwd_mma(const FwdParams& p, uint8_t* smem, FwdBarriers* b, uint3
     if (!fwd_item_exists<CAUSAL>(p, snake_unit(it >> 1, p.n_units), it & 1)) continue;
     if (!wait1(&b->q_full, qc & 1, b, p.status)) return;
     const int nk0 = *(volatile int*)&b->unit_nk[qc & 1][0];
-    const int nk1 = *(volatile int*)&b->unit_nk[qc & 1][1], nk = nk1;
+    const int nk1 = *(volatile int*)&b->unit_nk[qc & 1][1], nk = max(nk0, nk1);
     ++qc;
     tc_fence_after();
     for (int j = 0; j < nk; ++j) {
@@ -566,6 +568,7 @@ __device__ void fwd_softmax(const FwdParams& p, FwdBarriers* b, uint32_t tmem, i
       __syncwarp();
       if (lane_id() == 0) mbar_arrive(&b->p_full[wg]);  // one arrival per warp
     }
+    if (nk == 0) continue;  // a tile wholly past the last row: nothing to write
     // Epilogue: O = o / l, lse = (m + log2 l) ln 2.
     if (!wait_warp(&b->o_full[wg], oc & 1, b, p.status)) return;
     ++oc;
