@@ -284,6 +284,11 @@ int fa_gemm_tiles(int M, int N, int sms, int *tile_n, int *tiles_m, int *tiles_n
  */
 int fa_trace_start(void);
 int fa_trace_stop(int n_kernels, int *launches, double *total_ms);
+/* The same trace restricted to the kernels whose bit is set in kernel_mask
+ * (bit k: kernel id k); the others are launched without events, so a timed
+ * region can measure its dominant kernel while adding as few stream
+ * commands as possible.  fa_trace_start() is fa_trace_start_mask(~0u). */
+int fa_trace_start_mask(unsigned kernel_mask);
 const char *fa_trace_kernel_name(int kernel);
 
 /*

@@ -71,3 +71,8 @@ def test_public_calls_reject_bad_buffers_before_launch():
         with pytest.raises(ValueError):
             call()
             pytest.fail(f"case {i} was not rejected")
+
+
+def test_trace_start_rejects_unknown_kernel_names():
+    with pytest.raises(ValueError, match="unknown kernel"):
+        fa.trace_start(["fa_no_such_kernel"])

@@ -72,6 +72,7 @@ struct TraceRec {
 };
 std::mutex g_trace_mu;
 bool g_trace_on = false;
+unsigned g_trace_mask = 0;  // bit k set: kernel id k is bracketed
 std::vector<TraceRec> g_trace;
 std::vector<cudaEvent_t> g_event_pool[kMaxDevices];
 size_t g_event_used[kMaxDevices];
@@ -90,7 +91,7 @@ class LaunchTrace {
  public:
   LaunchTrace(int kernel, cudaStream_t s) : stream_(s) {
     std::lock_guard<std::mutex> lock(g_trace_mu);
-    if (!g_trace_on) return;
+    if (!g_trace_on || !((g_trace_mask >> kernel) & 1u)) return;
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return;
     rec_.kernel = kernel;
@@ -897,13 +898,16 @@ int fa_check_device_errors(fa_stream_t stream) {
   return FA_OK;
 }
 
-int fa_trace_start(void) {
+int fa_trace_start_mask(unsigned kernel_mask) {
   std::lock_guard<std::mutex> lock(g_trace_mu);
   g_trace.clear();
   for (int dev = 0; dev < kMaxDevices; ++dev) g_event_used[dev] = 0;
+  g_trace_mask = kernel_mask;
   g_trace_on = true;
   return FA_OK;
 }
+
+int fa_trace_start(void) { return fa_trace_start_mask(~0u); }
 
 int fa_trace_stop(int n_kernels, int* launches, double* total_ms) {
   std::lock_guard<std::mutex> lock(g_trace_mu);

@@ -30,7 +30,7 @@ EXPORTED = ["fa_fwd", "fa_bwd", "fa_bwd_workspace_size", "fa_strerror",
             "fa_trace_kernel_name", "fa_bwd_noalloc", "fa_bwd_deterministic",
             "fa_decode", "fa_decode_workspace_size", "fa_decode_plan", "fa_fwd_fp8",
             "fa_gemm", "fa_gemm_workspace_size", "fa_gemm_tiles", "fa_selftest_wait_timeout",
-            "fa_fwd_schedule"]
+            "fa_fwd_schedule", "fa_trace_start_mask"]
 NOALLOC_MAX_SCRATCH = 32 << 20  # FA_BWD_NOALLOC_MAX_SCRATCH
 KERNEL_IDS = {0: "fa_fwd_kernel", 1: "fa_bwd_prep", 2: "fa_bwd_kernel", 3: "unused",
               4: "fa_dq_kernel", 5: "fa_decode_kernel", 6: "fa_gemm_kernel", 7: "fa_gemm_pack"}
@@ -74,6 +74,8 @@ def load(path: str = LIB_PATH):
         lib.fa_launch_shape.restype = _i
         lib.fa_trace_start.argtypes = []
         lib.fa_trace_start.restype = _i
+        lib.fa_trace_start_mask.argtypes = [ctypes.c_uint]
+        lib.fa_trace_start_mask.restype = _i
         lib.fa_trace_stop.argtypes = [_i, ctypes.POINTER(_i), ctypes.POINTER(ctypes.c_double)]
         lib.fa_trace_stop.restype = _i
         lib.fa_trace_kernel_name.argtypes = [_i]
@@ -294,9 +296,19 @@ def launch_shape(pass_: int, B, H, N, d, causal=False):
     return ctas.value, units.value
 
 
-def trace_start() -> None:
-    """Start bracketing every library launch with CUDA events."""
-    _check(load().fa_trace_start(), "fa_trace_start")
+def trace_start(kernels=None) -> None:
+    """Start bracketing library launches with CUDA events: every launch, or
+    only those of the kernels named in `kernels` (names of KERNEL_IDS)."""
+    if kernels is None:
+        _check(load().fa_trace_start(), "fa_trace_start")
+        return
+    ids = {name: k for k, name in KERNEL_IDS.items()}
+    mask = 0
+    for name in kernels:
+        if name not in ids:
+            raise ValueError(f"unknown kernel {name!r}")
+        mask |= 1 << ids[name]
+    _check(load().fa_trace_start_mask(mask), "fa_trace_start_mask")
 
 
 def trace_stop() -> dict:
