@@ -36,8 +36,8 @@
 //               from TMEM through shared memory into the fp32 accumulator in
 //               global memory with bulk reduce-add copies.
 // Work units are ordered in groups of a few heads (so the dQ accumulator,
-// Q and dO of the heads in flight stay in L2), longest first (ascending K/V
-// block) within a group, and handed out dynamically.
+// Q and dO of the heads in flight stay in L2; bwd_group_heads), longest
+// first (ascending K/V block) within a group, and handed out dynamically.
 // TMEM columns: dV [0,D) dK [D,2D) S^T_s [2D+64s, +64) dP^T_s [2D+128+64s, +64)
 // for the two pipeline slots s; dQ^T of slot s overwrites dP^T_s once the
 // compute warps have read it, P^T_s (bf16 pairs) overwrites S^T_s.
@@ -63,8 +63,17 @@ inline size_t bwd_workspace_bytes(int B, int H, int N, int d) {
 }
 
 // Heads per scheduling group: the heads in flight keep their K, V, Q, dO and
-// dQ accumulator in L2.
-constexpr int kBwdGroupHeads = 8;
+// dQ accumulator in L2 (126 MB on B200).  The largest power of two up to 16
+// whose group needs at most 112 MB of it: per head N*d*12 bytes (four bf16
+// tensors and the fp32 accumulator).  More heads per group let the dynamic
+// scheduler balance the causal units' unequal lengths over more of them;
+// past the L2 budget the group's data no longer stays resident.
+inline int bwd_group_heads(int N, int d) {
+  const double per_head = static_cast<double>(N) * d * 12.0;
+  int g = 16;
+  while (g > 1 && g * per_head > 112.0 * (1 << 20)) g >>= 1;
+  return g;
+}
 
 struct BwdParams {
   void* dk;
@@ -79,6 +88,7 @@ struct BwdParams {
   int nq;       // ceil(N / 64) Q blocks
   int nkv;      // ceil(N / 128) K/V blocks
   int n_units;  // BH * nkv
+  int group_heads;  // heads per scheduling group (bwd_group_heads)
   float scale_log2;
   float scale;
   int grad_f32;
@@ -144,18 +154,19 @@ struct BwdUnit {
   int bh, j, i0, n;  // head, K/V block, first Q block, number of Q blocks
 };
 
-// Unit w -> (head, K/V block): groups of kBwdGroupHeads heads, K/V blocks in
+// Unit w -> (head, K/V block): groups of p.group_heads heads, K/V blocks in
 // ascending order within a group (the longest causal units first), heads
 // innermost.
 template <bool CAUSAL>
 __device__ __forceinline__ BwdUnit bwd_decode(const BwdParams& p, int w) {
   BwdUnit u;
-  const int per_group = kBwdGroupHeads * p.nkv;
+  const int gh = p.group_heads;
+  const int per_group = gh * p.nkv;
   const int g = w / per_group;
   const int r = w - g * per_group;
-  const int heads = min(kBwdGroupHeads, p.BH - g * kBwdGroupHeads);
+  const int heads = min(gh, p.BH - g * gh);
   u.j = r / heads;
-  u.bh = g * kBwdGroupHeads + (r - u.j * heads);
+  u.bh = g * gh + (r - u.j * heads);
   u.i0 = CAUSAL ? 2 * u.j : 0;
   u.n = p.nq - u.i0;
   return u;

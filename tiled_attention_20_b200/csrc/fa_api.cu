@@ -313,6 +313,7 @@ int launch_bwd(const void* q, const void* k, const void* v, const void* o, const
   p.nq = (N + 63) / 64;
   p.nkv = (N + 127) / 128;
   p.n_units = BH * p.nkv;
+  p.group_heads = fa::bwd_group_heads(N, d);
   p.scale_log2 = scale * 1.4426950408889634f;
   p.scale = scale;
   p.grad_f32 = grad_dtype;
