@@ -11,6 +11,8 @@ forward, halved when causal, and 2.5x that for the backward.
 Timing follows "第17讲 Tensor Core、HBM、SRAM 与 FlashAttention" §10.1-10.2:
 warm-up first, CUDA events on the launching stream with a synchronize on both
 sides, fixed shapes and dtypes, and a check of the outputs before timing.  The
+timed steps run as one CUDA graph (captured from the same library calls, which
+never allocate or synchronise), so the step time holds no host launch gaps.  The
 inputs and outputs of one step (about 0.6 GB) exceed the 126 MB L2, so no
 flush is needed between steps.
 
@@ -266,21 +268,37 @@ class ClockSampler:
 
 
 # ---------------------------------------------------------------- timing
+def graph_of(step, steps):
+    """One CUDA graph holding `steps` consecutive steps (every launch `step`
+    enqueues, captured on a side stream), replayed once untimed so that a
+    timed replay runs an instantiated, uploaded graph.  The library never
+    allocates or synchronises inside a call, so its launches capture as they
+    are; the graph removes the host launch gaps between the step's kernels."""
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, capture_error_mode="relaxed"):
+        for _ in range(steps):
+            step()
+    g.replay()
+    return g
+
+
 def timed_passes(step, steps, stream, dev, dist, world, quick=False, dominant=None):
-    """Timed passes of `step` on `stream`, each bracketed by a barrier and a
-    synchronize:
+    """Timed passes of `step`, each bracketed by a barrier and a synchronize.
+    Each pass captures its steps into one CUDA graph and times one replay of
+    it on `stream` (the warm-up steps ran as plain launches):
       1. the headline: `steps` steps between two CUDA events, with the
          launches of the `dominant` kernel (and only those, so the step gets
-         as few extra stream commands as possible) bracketed by events: its
-         duration for the roofline comes from the timed region itself;
+         as few extra nodes as possible) bracketed by external event nodes:
+         its duration for the roofline comes from the timed replay itself;
          returns the mean step time, max over ranks;
       2. the per-kernel table: `steps` steps with every library launch
-         bracketed by events;
-      3. the distribution: max(100, steps) steps with an event after each,
-         for the median, 10th and 90th percentile of the step time.
+         bracketed;
+      3. the distribution: max(100, steps) steps with an event node after
+         each, for the median, 10th and 90th percentile of the step time.
     Passes 2 and 3 run after the headline, when the power cap may have
-    lowered the clock.  With quick (profiler runs) only pass 1 runs, without
-    events.  Returns (mean ms, stats, dominant kernel's trace, all kernels)."""
+    lowered the clock.  With quick (profiler runs) only pass 1 runs, as plain
+    launches without events.  Returns (mean ms, stats, dominant kernel's
+    trace, all kernels)."""
     import tiled_attention_20_b200.fa as fa
 
     def sync():
@@ -288,35 +306,51 @@ def timed_passes(step, steps, stream, dev, dist, world, quick=False, dominant=No
             dist.barrier()
         torch.cuda.synchronize(dev)
 
-    sync()
     e0 = torch.cuda.Event(enable_timing=True)
     e1 = torch.cuda.Event(enable_timing=True)
-    if not quick:
-        fa.trace_start([dominant])
+    if quick:
+        sync()
+        e0.record(stream)
+        for _ in range(steps):
+            step()
+        e1.record(stream)
+        sync()
+        return ranks.max_over_ranks(e0.elapsed_time(e1) / steps, dist, dev), {}, {}, {}
+
+    fa.trace_start([dominant])
+    g = graph_of(step, steps)
+    sync()
     e0.record(stream)
-    for _ in range(steps):
-        step()
+    g.replay()
     e1.record(stream)
     sync()
-    dom = {} if quick else fa.trace_stop()
+    dom = fa.trace_stop()
     ms = ranks.max_over_ranks(e0.elapsed_time(e1) / steps, dist, dev)
-    if quick:
-        return ms, {}, dom, {}
+    del g
 
     fa.trace_start()
-    for _ in range(steps):
-        step()
+    g = graph_of(step, steps)
+    sync()
+    g.replay()
     sync()
     traced = fa.trace_stop()
+    del g
 
     n = max(100, steps)
-    ev = [torch.cuda.Event(enable_timing=True) for _ in range(n + 1)]
-    ev[0].record(stream)
-    for i in range(n):
-        step()
-        ev[i + 1].record(stream)
+    ev = [torch.cuda.Event(enable_timing=True, external=True) for _ in range(n + 1)]
+
+    def marked():
+        ev[0].record()
+        for i in range(n):
+            step()
+            ev[i + 1].record()
+
+    g = graph_of(marked, 1)
+    sync()
+    g.replay()
     sync()
     per = sorted(ev[i].elapsed_time(ev[i + 1]) for i in range(n))
+    del g
     pick = lambda f: per[min(n - 1, int(round(f * (n - 1))))]
     stats = {"n": n, "median_ms": statistics.median(per), "p10_ms": pick(0.1),
              "p90_ms": pick(0.9), "min_ms": per[0], "max_ms": per[-1],
@@ -642,7 +676,9 @@ def run_ours(args, rank, world, local_rank, dist):
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
             "dtype": "bf16", "data": "synthetic",
             "config": workload_config(w, {"parallelism": f"heads replicated per GPU x{world}",
-                                          "bwd": "deterministic" if args.deterministic else "atomic_dq"}),
+                                          "bwd": "deterministic" if args.deterministic else "atomic_dq",
+                                          "launch": "cuda_graph (each timed pass: its steps "
+                                                    "captured back to back, one replay timed)"}),
             "pct_of_peak": value / world / peaks["bf16_tflops"],
             "roofline": roof, "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": gpu_launches,
             "kernels": kernels, "clocks": clocks, "step_stats": stats,

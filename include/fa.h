@@ -280,7 +280,10 @@ int fa_gemm_tiles(int M, int N, int sms, int *tile_n, int *tiles_m, int *tiles_n
  * name).  The
  * library creates the events on first use and reuses them afterwards; event
  * records add a few microseconds per launch.  fa_trace_start() discards a
- * previous unfinished record.
+ * previous unfinished record.  Launches enqueued on a stream that is being
+ * captured into a CUDA graph are bracketed by external event nodes
+ * (cudaEventRecordExternal): the graph's replay stamps them, and
+ * fa_trace_stop() (called after the replay) reads the last replay's times.
  */
 int fa_trace_start(void);
 int fa_trace_stop(int n_kernels, int *launches, double *total_ms);

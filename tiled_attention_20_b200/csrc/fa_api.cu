@@ -58,7 +58,10 @@ EncodeTiledFn g_encode = nullptr;
 
 // ---------------------------------------------------------------- tracing
 // Opt-in per-kernel timing: while enabled, every launch is bracketed by a
-// pair of CUDA events on its stream.
+// pair of CUDA events on its stream.  On a stream that is being captured into
+// a CUDA graph the events are recorded as external event nodes, so every
+// replay of the graph stamps them (a plain record during capture would only
+// order the captured work).
 enum { kKernFwd = 0, kKernBwdPrep = 1, kKernBwd = 2, kKernBwdConvert = 3, kKernDq = 4,
        kKernDecode = 5, kKernGemm = 6, kKernGemmPack = 7, kNumKernels = 8 };
 const char* const kKernelNames[kNumKernels] = {"fa_fwd_kernel", "fa_bwd_prep", "fa_bwd_kernel",
@@ -98,17 +101,22 @@ class LaunchTrace {
     rec_.device = dev;
     rec_.start = trace_event(dev);
     rec_.stop = trace_event(dev);
-    if (rec_.start && rec_.stop && cudaEventRecord(rec_.start, s) == cudaSuccess) active_ = true;
+    cudaStreamCaptureStatus cap = cudaStreamCaptureStatusNone;
+    if (cudaStreamIsCapturing(s, &cap) != cudaSuccess) return;
+    flags_ = cap == cudaStreamCaptureStatusActive ? cudaEventRecordExternal : cudaEventRecordDefault;
+    if (rec_.start && rec_.stop && cudaEventRecordWithFlags(rec_.start, s, flags_) == cudaSuccess)
+      active_ = true;
   }
   ~LaunchTrace() {
     if (!active_) return;
     std::lock_guard<std::mutex> lock(g_trace_mu);
-    if (cudaEventRecord(rec_.stop, stream_) == cudaSuccess) g_trace.push_back(rec_);
+    if (cudaEventRecordWithFlags(rec_.stop, stream_, flags_) == cudaSuccess) g_trace.push_back(rec_);
   }
 
  private:
   cudaStream_t stream_;
   TraceRec rec_{};
+  unsigned flags_ = cudaEventRecordDefault;
   bool active_ = false;
 };
 
